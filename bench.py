@@ -1,0 +1,472 @@
+#!/usr/bin/env python
+"""Benchmark of one Muon optimizer step on B200: every Muon matrix of a parameter set
+in one grouped call (momentum, Nesterov input, Frobenius norm, 5 Newton-Schulz
+iterations, fused parameter update), timed with CUDA events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Under torchrun every rank steps its own copy of the
+parameter set (weak scaling, no collective on the data path); the step time is the
+maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from newton_schulz_11_b200 import inputs  # noqa: E402
+
+DEFAULT_WORKLOAD = "gpt2-124m-72-matrices"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KINDS = ("momentum", "norm", "gram", "poly", "apply", "apply_last")
+
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture of
+# the benchmarked workload, keyed by kernel kind; valid only while the kernel sources hash to
+# `source_hash` (see profiles/).  Filled in from the committed ncu summary.
+NCU_TRAFFIC = {"source_hash": None, "workload": DEFAULT_WORKLOAD, "bytes_per_launch": {}}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "newton_schulz_11_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ work model
+
+def matrix_work(rows, cols):
+    """Per matrix and iteration: algorithmic flops of the Gram (upper half), the
+    polynomial (upper half) and the apply, plus the dense-equivalent total."""
+    m, n = min(rows, cols), max(rows, cols)
+    return {"gram": m * m * n, "poly": m ** 3, "apply": 2 * m * m * n, "dense": 4 * m * m * n + 2 * m ** 3}
+
+
+def kind_bytes(w, kind, with_out=False):
+    """Algorithmic HBM bytes of one launch of `kind` over the whole workload."""
+    pb = 2 if w.param_dtype == "bf16" else 4
+    tot = 0
+    for rows, cols in w.shapes:
+        mn = rows * cols
+        m = min(rows, cols)
+        if kind == "momentum":
+            tot += 16 * mn           # read g, m; write m; write hi, lo
+        elif kind == "norm":
+            tot += 0
+        elif kind == "gram":
+            tot += 2 * mn + 2 * m * m
+        elif kind == "poly":
+            tot += 6 * m * m         # A operand, A in the epilogue, B out
+        elif kind == "apply":
+            tot += 10 * mn + 2 * m * m   # hi operand + hi, lo in, hi, lo out; B operand
+        elif kind == "apply_last":
+            tot += (6 + 2 * pb + (4 if with_out else 0)) * mn + 2 * m * m
+    return tot
+
+
+def kind_flops(w, kind):
+    if kind not in ("gram", "poly", "apply", "apply_last"):
+        return 0
+    key = "apply" if kind == "apply_last" else kind
+    return sum(matrix_work(r, c)[key] for r, c in w.shapes)
+
+
+def step_flops(w):
+    alg = sum(sum(matrix_work(r, c)[k] for k in ("gram", "poly", "apply")) for r, c in w.shapes) * w.ns_steps
+    dense = sum(matrix_work(r, c)["dense"] for r, c in w.shapes) * w.ns_steps
+    return alg, dense
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="muon_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def mark(self, begin: bool):
+        if begin:
+            self.t0 = datetime.datetime.now()
+        else:
+            self.t1 = datetime.datetime.now()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
+                except ValueError:
+                    continue
+                rows.append((ts, parts))
+        os.unlink(self.path)
+        inside = [p for ts, p in rows if self.t0 and self.t1 and self.t0 <= ts <= self.t1]
+        use = inside or [p for _, p in rows]
+        sm = [float(p[1]) for p in use if p[1].replace(".", "").isdigit()]
+        mx = [float(p[2]) for p in use if p[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for p in use:
+            for name, v in zip(names, p[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(use), "samples_in_timed_region": len(inside)}
+
+
+def gpu_id_for(device_index):
+    import torch
+
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid).replace("GPU-", "")
+    except Exception:  # pragma: no cover
+        return str(device_index)
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+
+def oracle_sample_ms(w, reps=1):
+    """Times the fp64 oracle on one matrix of each distinct shape and scales by the count
+    of that shape: milliseconds per full step (extrapolated), plus the sample description."""
+    import numpy as np
+
+    import oracle
+
+    coeffs = load_coeffs(w)
+    shapes = {}
+    for i, s in enumerate(w.shapes):
+        shapes.setdefault(s, []).append(i)
+    total_ms = 0.0
+    for s, idx in shapes.items():
+        i = idx[0]
+        step = inputs.first_step_index(w)
+        g = inputs.grad_np(w, step, i).astype(np.float64)
+        m = inputs.momentum_np(w, i).astype(np.float64)
+        W = inputs.weight_np(w, i).astype(np.float64)
+        best = float("inf")
+        for _ in range(reps):
+            t0 = time.perf_counter()
+            oracle.muon_step(W, g, m, lr=w.lr, beta=w.beta, weight_decay=w.weight_decay,
+                             nesterov=w.nesterov, coeffs=coeffs)
+            best = min(best, time.perf_counter() - t0)
+        total_ms += best * 1e3 * len(idx)
+    sample = (f"one matrix of each of the {len(shapes)} shapes of {w.name} through the fp64 oracle "
+              f"(momentum, NS x{w.ns_steps}, update), time scaled by the count of each shape")
+    return total_ms, sample
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:  # pragma: no cover
+        return os.cpu_count()
+
+
+def load_coeffs(w):
+    from newton_schulz_11_b200 import schedules
+
+    if w.schedule == "polar5":
+        return schedules.load("polar5")
+    return [(3.4445, -4.7750, 2.0315)] * w.ns_steps
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def dist_max(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args, world, rank):
+    """The oracle, as it stands, on the host cores: each step is one bounded sample of the
+    workload (one matrix per shape), scaled to a full step."""
+    if rank != 0:
+        return
+    w = inputs.WORKLOADS[args.workload]
+    for _ in range(args.warmup):
+        oracle_sample_ms(w)
+    runs = [oracle_sample_ms(w) for _ in range(args.steps)]
+    sample = runs[0][1]
+    value = statistics.median(r[0] for r in runs)
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": "muon_step_ms", "value": round(value, 3), "unit": "ms",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(value, 3),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name, "matrices": len(w.shapes), "params": w.n_params},
+        "cpu_baseline": {"value": round(value, 3), "unit": "ms", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, world, rank, local):
+    import ctypes
+
+    import torch
+
+    from newton_schulz_11_b200 import _lib, api, build
+
+    build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = inputs.WORKLOADS[args.workload]
+    coeffs = load_coeffs(w)
+    step0 = inputs.first_step_index(w)
+
+    # flat device buffers with one 2-D view per matrix (one H2D / D2H copy per step in e2e)
+    sizes = [r * c for r, c in w.shapes]
+    offs = [0]
+    for s in sizes:
+        offs.append(offs[-1] + s)
+    pdt = torch.bfloat16 if w.param_dtype == "bf16" else torch.float32
+    G = torch.empty(offs[-1], dtype=torch.float32, device=dev)
+    M = torch.empty(offs[-1], dtype=torch.float32, device=dev)
+    P = torch.empty(offs[-1], dtype=pdt, device=dev)
+    view = lambda flat, i: flat[offs[i]: offs[i + 1]].view(*w.shapes[i])  # noqa: E731
+    gs = [view(G, i) for i in range(len(sizes))]
+    ms = [view(M, i) for i in range(len(sizes))]
+    ps = [view(P, i) for i in range(len(sizes))]
+    with torch.no_grad():
+        for i in range(len(sizes)):
+            gs[i].copy_(inputs.grad_torch(w, step0, i, dev))
+            ms[i].copy_(inputs.momentum_torch(w, i, dev))
+            ps[i].copy_(inputs.weight_torch(w, i, dev))
+    torch.cuda.synchronize()
+
+    ws = api.Workspace(dev)
+    stream = torch.cuda.current_stream(dev)
+    kw = dict(lr=w.lr, beta=w.beta, weight_decay=w.weight_decay, nesterov=w.nesterov, coeffs=coeffs,
+              workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        api.muon_step(ps, gs, ms, **kw)
+    torch.cuda.synchronize()
+
+    L = _lib.lib()
+    clocks = ClockSampler(gpu_id_for(local))
+    clocks.start()
+    # ---- timed region: K steps, inputs resident in HBM (larger than L2)
+    barrier(world)
+    torch.cuda.synchronize()
+    _lib.check(L.muon_profile_begin(), "muon_profile_begin")
+    clocks.mark(True)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        api.muon_step(ps, gs, ms, **kw)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark(False)
+    barrier(world)
+    kms = (ctypes.c_double * 6)()
+    kcount = (ctypes.c_int64 * 6)()
+    _lib.check(L.muon_profile_end(kms, kcount, 6), "muon_profile_end")
+    ms_step = e0.elapsed_time(e1) / args.steps
+    clk = clocks.stop()
+    ms_step = dist_max(ms_step, world)
+
+    # ---- end to end through host buffers: H2D grads, step, D2H params, every step
+    pin_g = torch.empty_like(G, device="cpu").pin_memory()
+    pin_g.copy_(G.cpu())
+    pin_p = torch.empty_like(P, device="cpu").pin_memory()
+    for _ in range(2):
+        G.copy_(pin_g, non_blocking=True)
+        api.muon_step(ps, gs, ms, **kw)
+        pin_p.copy_(P, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, min(args.steps, 50))
+    f0.record(stream)
+    for _ in range(e2e_steps):
+        G.copy_(pin_g, non_blocking=True)
+        api.muon_step(ps, gs, ms, **kw)
+        pin_p.copy_(P, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = dist_max(f0.elapsed_time(f1) / e2e_steps, world)
+    barrier(world)
+
+    code, where = api.device_status(ws)
+    if code != 0:
+        raise RuntimeError(f"device status {code} at wait site {where}")
+
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    per_kind = {k: {"ms_total": kms[i], "launches": int(kcount[i])} for i, k in enumerate(KINDS)}
+    dom = max(KINDS, key=lambda k: per_kind[k]["ms_total"])
+    dom_launches = max(1, per_kind[dom]["launches"])
+    dom_ms = per_kind[dom]["ms_total"] / dom_launches
+    fl = kind_flops(w, dom)
+    by = kind_bytes(w, dom)
+    tf = fl / (dom_ms * 1e-3) / 1e12 if fl else 0.0
+    gbs = by / (dom_ms * 1e-3) / 1e9
+    f_tensor = tf / peaks["bf16_tflops"] if fl else 0.0
+    f_hbm = gbs / peaks["hbm_gbs"]
+    traffic = None
+    if NCU_TRAFFIC["source_hash"] == kernel_source_hash() and NCU_TRAFFIC["workload"] == w.name:
+        traffic = NCU_TRAFFIC["bytes_per_launch"].get(dom)
+    if f_tensor >= f_hbm:
+        roof = {"bound": "tensor", "achieved": round(tf, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(f_tensor, 4)}
+    else:
+        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(f_hbm, 4)}
+    roof.update({"traffic": traffic, "kernel": dom, "peak_source": peak_src,
+                 "other_bound_frac": round(min(f_tensor, f_hbm), 4),
+                 "algorithmic_bytes_per_launch": by, "algorithmic_flops_per_launch": fl,
+                 "ms_per_launch": round(dom_ms, 4)})
+
+    alg, dense = step_flops(w)
+    line = {
+        "metric": "muon_step_ms", "value": round(ms_step, 4), "unit": "ms", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "matrices": len(w.shapes), "params": w.n_params,
+                   "param_dtype": w.param_dtype, "ns_steps": w.ns_steps, "schedule": w.schedule,
+                   "l2": "inputs larger than L2 (grads+momentum+params ~%.2f GB)" % (w.n_params * 10 / 1e9),
+                   "parallelism": "replicas" if world > 1 else "single"},
+        "ns_tflops": round(world * alg / (ms_step * 1e-3) / 1e12, 1),
+        "ns_tflops_dense_equiv": round(world * dense / (ms_step * 1e-3) / 1e12, 1),
+        "ns_frac_of_bf16_peak": round(alg / (ms_step * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+        "kernels": {k: {"ms_per_launch": round(v["ms_total"] / max(1, v["launches"]), 4),
+                        "launches": v["launches"], "share": round(v["ms_total"] / max(1e-9, sum(
+                            x["ms_total"] for x in per_kind.values())), 4)} for k, v in per_kind.items()},
+        "roofline": roof,
+        "clocks": clk,
+        "e2e": {"value": round(e2e_ms, 4), "unit": "ms", "h2d_bytes_per_step": G.numel() * 4,
+                "d2h_bytes_per_step": P.numel() * P.element_size()},
+        "gpu_launches": int(sum(kcount)),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        cms, sample = oracle_sample_ms(w)
+        line["cpu_baseline"] = {"value": round(cms, 1), "unit": "ms", "cores": blas_threads(), "kind": "oracle",
+                                "sample": sample}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=inputs.WORKLOAD_ORDER)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup(args)
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,190 @@
+/*
+ * muon_b200.h -- C ABI of the B200 (sm_100a) Muon optimizer step.
+ *
+ * The operation, as the pages define it:
+ *
+ *   momentum  m <- beta * m + g
+ *             ("14 - modded-nanogpt: the Speedrun Community", section 3 "Muon",
+ *              muon_step pseudocode)
+ *   Nesterov  u = g + beta * m   (nesterov != 0), else u = m
+ *             ("NanoGPT Speedrun" README, practices list after the Newton-Schulz
+ *              listing: Nesterov momentum inside the update, orthogonalisation after
+ *              the momentum; the page's full formula was lost, this is the reading)
+ *   NS        X = u / (||u||_F + eps), short side on the rows, then per iteration k
+ *             A = X X^T,  B = b_k A + c_k A A,  X = a_k X + B X,  transpose back
+ *             ("NanoGPT Speedrun" README, zeroth_power_via_newtonschulz5 listing;
+ *              a row per iteration covers the "Polar Express" schedules named in the
+ *              same README's technique list)
+ *   update    W <- W (1 - lr * wd) - lr * shape_scale * O
+ *             (decoupled weight decay from the old W; the README's record list names
+ *              "standard weight decay" and "Muon custom sizing" without formulas)
+ *
+ * Layout: every matrix is row-major, element (r, c) at base + r * ld + c, with
+ * ld >= cols counted in elements.  Gradients and momentum are fp32; the parameter
+ * is fp32 or bf16; the optional O output is dense fp32 (ld = cols).
+ *
+ * Ownership: the caller allocates and owns every buffer, including the workspace,
+ * and keeps them alive until the work queued on `stream` has finished.  The library
+ * allocates no device memory.  `param` and `momentum` are updated in place; `grad`
+ * is only read.  Buffers of different roles (and of different matrices) must not
+ * overlap.  All device pointers must belong to the current CUDA device.
+ *
+ * Execution: asynchronous on `stream` (a cudaStream_t; NULL is the legacy default
+ * stream).  No call synchronises the host except muon_device_status.  The first
+ * call with a new set of descriptors plans the work (host only, microseconds) and
+ * caches the plan; later calls with identical descriptors reuse it.
+ *
+ * Errors: every entry point returns a muon_status_t.  On a validation error
+ * nothing is launched and no buffer is touched.  A failed CUDA launch returns
+ * MUON_ERR_CUDA.  Device-side waits are bounded: a wait that runs out records
+ * MUON_ERR_TIMEOUT in the workspace's status word (read it with
+ * muon_device_status) and the kernel returns instead of hanging.
+ *
+ * Numerics: Newton-Schulz runs with bf16 tensor-core operands and fp32
+ * accumulation; X is carried between iterations as a bf16 pair (hi + lo), which
+ * holds about 16 significant bits, so that the a*X term does not lose the
+ * precision a single bf16 copy would.  Momentum and the update are fp32.
+ * Finite inputs with ||u||_F below about 1e17 are required (the Gram of the
+ * unscaled bf16 input is formed before the 1/||u||^2 factor is applied).
+ */
+#ifndef MUON_B200_H
+#define MUON_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MUON_ABI_VERSION 1
+#define MUON_MAX_NS_STEPS 16
+
+typedef enum {
+  MUON_OK = 0,
+  MUON_ERR_INVALID_ARG = 1,        /* null pointer, n < 1, bad hyperparameter, overlap */
+  MUON_ERR_ALIGNMENT = 2,          /* a pointer is not aligned to its element size */
+  MUON_ERR_UNSUPPORTED_SHAPE = 3,  /* rows/cols < 1, ld < cols, or a side above 2^24 */
+  MUON_ERR_UNSUPPORTED_DTYPE = 4,  /* param_dtype not MUON_F32 / MUON_BF16 */
+  MUON_ERR_WORKSPACE_TOO_SMALL = 5,/* not even the largest single matrix fits */
+  MUON_ERR_CUDA = 6,               /* a CUDA runtime call or launch failed */
+  MUON_ERR_TIMEOUT = 7,            /* device status only: a bounded wait ran out */
+  MUON_ERR_NO_DEVICE = 8           /* current device is not an sm_100 GPU */
+} muon_status_t;
+
+typedef enum { MUON_F32 = 0, MUON_BF16 = 1 } muon_dtype_t;
+
+/* One 2-D parameter.  80 bytes, no implicit padding. */
+typedef struct {
+  void*        param;        /* in/out: W, param_dtype, [rows x ld_param]; may be NULL
+                                only in muon_newton_schulz */
+  const float* grad;         /* in: g (muon_step) or G (muon_newton_schulz), fp32 [rows x ld_grad] */
+  float*       momentum;     /* in/out: m, fp32 [rows x ld_mom]; ignored by muon_newton_schulz */
+  float*       out_update;   /* optional out: O = NS(u), dense fp32 [rows x cols]; NULL skips it */
+  int64_t      rows;
+  int64_t      cols;
+  int64_t      ld_param;     /* row stride of param, elements */
+  int64_t      ld_grad;      /* row stride of grad, elements */
+  int64_t      ld_mom;       /* row stride of momentum, elements */
+  int32_t      param_dtype;  /* muon_dtype_t */
+  float        shape_scale;  /* multiplier on lr; <= 0 selects sqrt(max(1, rows / cols)) */
+} muon_matrix_t;
+
+/* Where one matrix's scratch lives inside the workspace (diagnostics and tests). */
+typedef struct {
+  uint64_t x_hi_offset[2];   /* bf16 [rows x x_ld]: ping-pong high parts of X */
+  uint64_t x_lo_offset;      /* bf16 [rows x x_ld]: low part of X */
+  uint64_t a_offset;         /* bf16 [m x a_ld]: A = X X^T of the latest iteration */
+  uint64_t b_offset;         /* bf16 [m x a_ld]: B = b A + c A A of the latest iteration */
+  uint64_t scale_offset;     /* fp32: 1 / (||u||_F + eps) */
+  uint64_t norm_offset;      /* fp32: ||u||_F */
+  int64_t  x_ld;             /* elements */
+  int64_t  a_ld;             /* elements */
+  int32_t  wave;             /* matrices are processed in waves that reuse the workspace */
+  int32_t  transposed;       /* 1 when rows > cols (X is the transpose of the stored matrix) */
+} muon_scratch_view_t;
+
+/* Version of this ABI (MUON_ABI_VERSION of the library that was loaded). */
+int muon_abi_version(void);
+
+/* Static, human-readable text for a status code. */
+const char* muon_status_str(int status);
+
+/*
+ * Bytes of workspace that lets muon_step / muon_newton_schulz process all n
+ * matrices at full speed.  A smaller workspace is accepted as long as the
+ * largest single matrix fits; the matrices are then processed in more waves.
+ */
+muon_status_t muon_workspace_size(const muon_matrix_t* mats, int n, size_t* bytes);
+
+/*
+ * Zeroes the device status word at the start of a workspace (queued on `stream`).
+ * Call once after allocating a workspace; the word is sticky until cleared again.
+ */
+muon_status_t muon_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * One Muon step on n matrices (one grouped launch sequence).
+ *   lr, beta, weight_decay : finite; beta in [0, 1]; lr >= 0; weight_decay >= 0
+ *   nesterov               : 0 or 1
+ *   ns_steps, coeffs       : 1 <= ns_steps <= MUON_MAX_NS_STEPS; coeffs is a HOST array of
+ *                            ns_steps rows (a, b, c), row k used in iteration k
+ *   eps                    : added to the Frobenius norm (the page uses 1e-7); > 0
+ *   workspace              : device memory, 256-byte aligned, from muon_workspace_size
+ */
+muon_status_t muon_step(const muon_matrix_t* mats, int n, float lr, float beta,
+                        float weight_decay, int nesterov, int ns_steps, const float* coeffs,
+                        float eps, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Newton-Schulz alone (zeroth_power_via_newtonschulz5 with a coefficient table):
+ * reads mats[i].grad as G and writes NS(G) to mats[i].out_update (required here).
+ * param and momentum are ignored and left untouched.
+ */
+muon_status_t muon_newton_schulz(const muon_matrix_t* mats, int n, int ns_steps,
+                                 const float* coeffs, float eps, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/* Scratch placement of matrix `index` for this descriptor set and workspace size. */
+muon_status_t muon_scratch_view(const muon_matrix_t* mats, int n, int index,
+                                size_t workspace_bytes, muon_scratch_view_t* view);
+
+/*
+ * Waits for `stream`, then reads the workspace's device status word into
+ * *device_status (MUON_OK or MUON_ERR_TIMEOUT) and *where (the wait that gave up).
+ */
+muon_status_t muon_device_status(const void* workspace, void* stream, int32_t* device_status,
+                                 int32_t* where);
+
+/*
+ * Budget of every device-side wait, in microseconds (default 2,000,000 = 2 s).  A
+ * value <= 0 restores the default.  Takes effect for launches queued afterwards.
+ * Waits on the way out of a kernel that gave up (for copies and MMAs already in
+ * flight) always get at least 2 s.
+ */
+muon_status_t muon_set_wait_timeout_us(int64_t us);
+
+/*
+ * Per-kernel timing for diagnostics and benchmarks.  Between muon_profile_begin and
+ * muon_profile_end every launch the library queues is bracketed by a pair of CUDA
+ * events recorded on its own stream.  muon_profile_end waits for those events and
+ * returns, per kernel kind (MUON_KIND_*), the summed device time in milliseconds and
+ * the number of launches.  Timing state is per process; calls are not thread safe
+ * while a profile is open.
+ */
+#define MUON_KIND_MOMENTUM 0   /* momentum, Nesterov input, hi/lo split, chunk sums */
+#define MUON_KIND_NORM 1       /* per-matrix norm and scale */
+#define MUON_KIND_GRAM 2       /* A = X X^T */
+#define MUON_KIND_POLY 3       /* B = b A + c A A */
+#define MUON_KIND_APPLY 4      /* X <- a X + B X */
+#define MUON_KIND_APPLY_LAST 5 /* last iteration, fused parameter update */
+#define MUON_NUM_KINDS 6
+
+muon_status_t muon_profile_begin(void);
+muon_status_t muon_profile_end(double* ms_by_kind, int64_t* launches_by_kind, int kinds);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUON_B200_H */

@@ -1,0 +1,201 @@
+"""PyTorch-facing binding: turns tensors into muon_matrix_t descriptors and calls the C ABI.
+
+Only argument marshalling happens here; every step of the Muon update runs in
+libmuon_b200.so.  PyTorch provides the device memory and the current stream.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import List, Optional, Sequence, Tuple
+
+import torch
+
+from . import _lib
+from ._lib import MuonError, MuonLibraryError, MuonMatrix, MuonScratchView, check, lib  # noqa: F401
+
+# "NanoGPT Speedrun" README, zeroth_power_via_newtonschulz5 listing: (a, b, c), 5 steps, eps.
+QUINTIC = (3.4445, -4.7750, 2.0315)
+DEFAULT_STEPS = 5
+DEFAULT_EPS = 1e-7
+
+
+def quintic_table(steps: int = DEFAULT_STEPS) -> List[Tuple[float, float, float]]:
+    return [QUINTIC] * steps
+
+
+def _coeff_array(coeffs) -> Tuple[ctypes.Array, int]:
+    rows = [tuple(float(v) for v in r) for r in coeffs]
+    if not rows or any(len(r) != 3 for r in rows):
+        raise ValueError("coeffs must be a non-empty sequence of (a, b, c) rows")
+    flat = (ctypes.c_float * (3 * len(rows)))(*[v for r in rows for v in r])
+    return flat, len(rows)
+
+
+def _check_2d(t: torch.Tensor, what: str, dtypes) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{what} must be a torch.Tensor")
+    if t.dim() != 2:
+        raise ValueError(f"{what} must be 2-D (Muon orthogonalises matrices only), got shape {tuple(t.shape)}")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{what} has dtype {t.dtype}, expected one of {dtypes}")
+    if not t.is_cuda:
+        raise ValueError(f"{what} must live on a CUDA device")
+    if t.stride(1) != 1 and t.shape[1] > 1:
+        raise ValueError(f"{what} must have unit stride along its last dimension")
+
+
+def _ld(t: torch.Tensor) -> int:
+    return t.stride(0) if t.shape[0] > 1 else t.shape[1]
+
+
+def _descriptors(params, grads, moms, outs, shape_scales, ns_only: bool) -> ctypes.Array:
+    n = len(grads)
+    arr = (MuonMatrix * n)()
+    dev = grads[0].device
+    for i in range(n):
+        g = grads[i]
+        _check_2d(g, f"grads[{i}]", (torch.float32,))
+        if g.device != dev:
+            raise ValueError("all tensors must be on the same device")
+        d = arr[i]
+        d.rows, d.cols = g.shape
+        d.grad = g.data_ptr()
+        d.ld_grad = _ld(g)
+        d.shape_scale = 0.0 if shape_scales is None or shape_scales[i] is None else float(shape_scales[i])
+        if outs is not None and outs[i] is not None:
+            o = outs[i]
+            _check_2d(o, f"outs[{i}]", (torch.float32,))
+            if tuple(o.shape) != tuple(g.shape) or not o.is_contiguous():
+                raise ValueError(f"outs[{i}] must be a contiguous fp32 tensor of shape {tuple(g.shape)}")
+            d.out_update = o.data_ptr()
+        if ns_only:
+            d.param_dtype = _lib.MUON_F32
+            continue
+        p, m = params[i], moms[i]
+        _check_2d(p, f"params[{i}]", (torch.float32, torch.bfloat16))
+        _check_2d(m, f"moms[{i}]", (torch.float32,))
+        if tuple(p.shape) != tuple(g.shape) or tuple(m.shape) != tuple(g.shape):
+            raise ValueError(f"params[{i}], grads[{i}] and moms[{i}] must have the same shape")
+        if p.device != dev or m.device != dev:
+            raise ValueError("all tensors must be on the same device")
+        d.param = p.data_ptr()
+        d.param_dtype = _lib.MUON_BF16 if p.dtype == torch.bfloat16 else _lib.MUON_F32
+        d.ld_param = _ld(p)
+        d.momentum = m.data_ptr()
+        d.ld_mom = _ld(m)
+    return arr
+
+
+class Workspace:
+    """Device scratch owned by the caller (PyTorch memory), grown on demand, one per device."""
+
+    def __init__(self, device):
+        self.device = torch.device(device)
+        self.buf: Optional[torch.Tensor] = None
+
+    @property
+    def nbytes(self) -> int:
+        return 0 if self.buf is None else self.buf.numel()
+
+    def ensure(self, nbytes: int, stream: int) -> Tuple[int, int]:
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = None
+            self.buf = torch.empty(int(nbytes), dtype=torch.uint8, device=self.device)
+            check(lib().muon_workspace_init(self.buf.data_ptr(), self.buf.numel(), stream), "muon_workspace_init")
+        return self.buf.data_ptr(), self.buf.numel()
+
+
+_workspaces = {}
+
+
+def default_workspace(device) -> Workspace:
+    device = torch.device(device)
+    key = device.index if device.index is not None else torch.cuda.current_device()
+    ws = _workspaces.get(key)
+    if ws is None:
+        ws = _workspaces[key] = Workspace(torch.device("cuda", key))
+    return ws
+
+
+def workspace_size(shapes: Sequence[Tuple[int, int]]) -> int:
+    n = len(shapes)
+    arr = (MuonMatrix * n)()
+    for i, (r, c) in enumerate(shapes):
+        arr[i].rows, arr[i].cols = int(r), int(c)
+    out = ctypes.c_size_t(0)
+    check(lib().muon_workspace_size(arr, n, ctypes.byref(out)), "muon_workspace_size")
+    return int(out.value)
+
+
+def _stream_handle(device, stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return int(stream.cuda_stream)
+
+
+def muon_step(params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor], moms: Sequence[torch.Tensor], *,
+              lr: float, beta: float = 0.95, weight_decay: float = 0.0, nesterov: bool = True,
+              coeffs=None, eps: float = DEFAULT_EPS, shape_scales=None, outs=None,
+              workspace: Optional[Workspace] = None, workspace_bytes: Optional[int] = None, stream=None) -> None:
+    """One grouped Muon step, in place on params and moms (see include/muon_b200.h).
+
+    ``outs`` (optional, fp32, same shapes) receives the orthogonalised update O.
+    ``workspace_bytes`` caps the scratch used (fewer bytes -> more waves).
+    """
+    if not (len(params) == len(grads) == len(moms)) or len(grads) == 0:
+        raise ValueError("params, grads and moms must be equally long, non-empty lists")
+    table, steps = _coeff_array(coeffs if coeffs is not None else quintic_table())
+    device = grads[0].device
+    arr = _descriptors(params, grads, moms, outs, shape_scales, ns_only=False)
+    n = len(grads)
+    h = lib()
+    need = ctypes.c_size_t(0)
+    check(h.muon_workspace_size(arr, n, ctypes.byref(need)), "muon_workspace_size")
+    s = _stream_handle(device, stream)
+    ws = workspace or default_workspace(device)
+    want = int(need.value) if workspace_bytes is None else int(workspace_bytes)
+    ptr, size = ws.ensure(want, s)
+    check(h.muon_step(arr, n, float(lr), float(beta), float(weight_decay), 1 if nesterov else 0, steps, table,
+                      float(eps), ptr, min(size, want), s), "muon_step")
+
+
+def newton_schulz(Gs: Sequence[torch.Tensor], *, coeffs=None, eps: float = DEFAULT_EPS, outs=None,
+                  workspace: Optional[Workspace] = None, workspace_bytes: Optional[int] = None,
+                  stream=None) -> List[torch.Tensor]:
+    """zeroth_power_via_newtonschulz5 on each fp32 matrix of Gs, grouped; returns fp32 O's."""
+    Gs = list(Gs)
+    if not Gs:
+        raise ValueError("Gs must be a non-empty list")
+    if outs is None:
+        outs = [torch.empty_like(g) for g in Gs]
+    table, steps = _coeff_array(coeffs if coeffs is not None else quintic_table())
+    device = Gs[0].device
+    arr = _descriptors(None, Gs, None, outs, None, ns_only=True)
+    n = len(Gs)
+    h = lib()
+    need = ctypes.c_size_t(0)
+    check(h.muon_workspace_size(arr, n, ctypes.byref(need)), "muon_workspace_size")
+    s = _stream_handle(device, stream)
+    ws = workspace or default_workspace(device)
+    want = int(need.value) if workspace_bytes is None else int(workspace_bytes)
+    ptr, size = ws.ensure(want, s)
+    check(h.muon_newton_schulz(arr, n, steps, table, float(eps), ptr, min(size, want), s), "muon_newton_schulz")
+    return outs
+
+
+def scratch_view(shapes: Sequence[Tuple[int, int]], index: int, workspace_bytes: int) -> MuonScratchView:
+    n = len(shapes)
+    arr = (MuonMatrix * n)()
+    for i, (r, c) in enumerate(shapes):
+        arr[i].rows, arr[i].cols = int(r), int(c)
+    v = MuonScratchView()
+    check(lib().muon_scratch_view(arr, n, int(index), int(workspace_bytes), ctypes.byref(v)), "muon_scratch_view")
+    return v
+
+
+def device_status(workspace: Workspace, stream=None) -> Tuple[int, int]:
+    code, where = ctypes.c_int32(0), ctypes.c_int32(0)
+    s = _stream_handle(workspace.device, stream)
+    check(lib().muon_device_status(workspace.buf.data_ptr(), s, ctypes.byref(code), ctypes.byref(where)),
+          "muon_device_status")
+    return int(code.value), int(where.value)

@@ -1,0 +1,142 @@
+// Elementwise stage of the Muon step, HBM-bound.
+//
+//   m' = beta m + g                        ("14 - modded-nanogpt", section 3, muon_step)
+//   u  = g + beta m'  (Nesterov) or m'     ("NanoGPT Speedrun" README, practices list)
+//   hi = bf16(u), lo = bf16(u - hi)        Newton-Schulz input, unscaled
+//   partial[chunk] = sum of u^2            for ||u||_F of the listing's G.norm()
+//
+// followed by a per-matrix finalisation s = 1 / (||u||_F + eps) in a fixed order
+// (deterministic: no atomics).  One CTA handles one chunk of whole rows of one
+// matrix; rows are read with 128-bit loads when the layout allows it.
+#include "muon_device.cuh"
+#include "muon_params.h"
+
+namespace muon {
+
+constexpr int kEwThreads = 256;
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float s = 0.f;
+  if (warp == 0) {
+    s = lane < (kEwThreads / 32) ? red[lane] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  }
+  return s;  // valid in thread 0
+}
+
+__device__ __forceinline__ int find_matrix(const EwParams& p, int chunk) {
+  int lo = 0, hi = p.n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.mats[mid].chunk_begin <= chunk) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ float ew_one(float g, float& m, float beta, int nesterov, int ns_only) {
+  if (ns_only) return g;
+  const float mn = fmaf(beta, m, g);
+  m = mn;
+  return nesterov ? fmaf(beta, mn, g) : mn;
+}
+
+__global__ void __launch_bounds__(kEwThreads) muon_momentum_kernel(const __grid_constant__ EwParams p) {
+  __shared__ float red[kEwThreads / 32];
+  const int chunk = blockIdx.x;
+  const int i = find_matrix(p, chunk);
+  const EwMat& t = p.mats[i];
+  const int r0 = (chunk - t.chunk_begin) * t.rows_per_chunk;
+  const int r1 = min(t.rows, r0 + t.rows_per_chunk);
+  const float beta = p.beta;
+  const int nesterov = p.nesterov, ns_only = p.ns_only;
+  float acc = 0.f;
+
+  if (t.vec) {
+    const int c4 = t.cols >> 2;
+    const int total = (r1 - r0) * c4;
+    for (int idx = threadIdx.x; idx < total; idx += kEwThreads) {
+      const int rr = idx / c4;
+      const int c = (idx - rr * c4) << 2;
+      const int r = r0 + rr;
+      const float4 g = __ldcs(reinterpret_cast<const float4*>(t.g + static_cast<int64_t>(r) * t.ld_g + c));
+      float4 m = make_float4(0.f, 0.f, 0.f, 0.f);
+      float* mp = t.m + static_cast<int64_t>(r) * t.ld_m + c;
+      if (!ns_only) m = __ldcs(reinterpret_cast<const float4*>(mp));
+      float u0 = ew_one(g.x, m.x, beta, nesterov, ns_only);
+      float u1 = ew_one(g.y, m.y, beta, nesterov, ns_only);
+      float u2 = ew_one(g.z, m.z, beta, nesterov, ns_only);
+      float u3 = ew_one(g.w, m.w, beta, nesterov, ns_only);
+      if (!ns_only) __stcs(reinterpret_cast<float4*>(mp), m);
+      uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
+      split_hi_lo(u0, h0, l0);
+      split_hi_lo(u1, h1, l1);
+      split_hi_lo(u2, h2, l2);
+      split_hi_lo(u3, h3, l3);
+      const int64_t o = static_cast<int64_t>(r) * t.ldx + c;
+      *reinterpret_cast<uint2*>(t.hi + o) = make_uint2(h0 | (h1 << 16), h2 | (h3 << 16));
+      *reinterpret_cast<uint2*>(t.lo + o) = make_uint2(l0 | (l1 << 16), l2 | (l3 << 16));
+      acc = fmaf(u0, u0, acc);
+      acc = fmaf(u1, u1, acc);
+      acc = fmaf(u2, u2, acc);
+      acc = fmaf(u3, u3, acc);
+    }
+  } else {
+    const int total = (r1 - r0) * t.cols;
+    for (int idx = threadIdx.x; idx < total; idx += kEwThreads) {
+      const int rr = idx / t.cols;
+      const int c = idx - rr * t.cols;
+      const int r = r0 + rr;
+      const float g = t.g[static_cast<int64_t>(r) * t.ld_g + c];
+      float* mp = t.m + static_cast<int64_t>(r) * t.ld_m + c;
+      float m = ns_only ? 0.f : *mp;
+      const float u = ew_one(g, m, beta, nesterov, ns_only);
+      if (!ns_only) *mp = m;
+      uint32_t h, l;
+      split_hi_lo(u, h, l);
+      const int64_t o = static_cast<int64_t>(r) * t.ldx + c;
+      t.hi[o] = __ushort_as_bfloat16(static_cast<unsigned short>(h));
+      t.lo[o] = __ushort_as_bfloat16(static_cast<unsigned short>(l));
+      acc = fmaf(u, u, acc);
+    }
+  }
+  const float s = block_sum(acc, red);
+  if (threadIdx.x == 0) p.partials[chunk] = s;
+}
+
+// s_i = 1 / (sqrt(sum of the matrix's chunk partials) + eps), summed in fp64 in a
+// fixed order.
+__global__ void __launch_bounds__(kEwThreads) muon_norm_kernel(const __grid_constant__ EwParams p) {
+  __shared__ double red[kEwThreads];
+  const EwMat& t = p.mats[blockIdx.x];
+  double s = 0.0;
+  for (int k = threadIdx.x; k < t.nchunks; k += kEwThreads) s += static_cast<double>(p.partials[t.chunk_begin + k]);
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = kEwThreads / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const double nrm = sqrt(red[0]);
+    p.norm[blockIdx.x] = static_cast<float>(nrm);
+    p.scale[blockIdx.x] = static_cast<float>(1.0 / (nrm + static_cast<double>(p.eps)));
+  }
+}
+
+cudaError_t launch_momentum(const EwParams& p, cudaStream_t stream) {
+  muon_momentum_kernel<<<p.total_chunks, kEwThreads, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_norm(const EwParams& p, cudaStream_t stream) {
+  muon_norm_kernel<<<p.n, kEwThreads, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace muon

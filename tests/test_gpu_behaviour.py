@@ -1,0 +1,137 @@
+"""Behaviour of the CUDA path beyond single-call parity: determinism, waves, strided
+views, NaN isolation between matrices, no-op on invalid calls, state round trip."""
+import numpy as np
+import pytest
+
+import oracle
+from newton_schulz_11_b200 import inputs
+from tests.gpu_util import rel_fro, require_gpu, to_np, torch
+
+pytestmark = pytest.mark.gpu
+QUINTIC5 = [oracle.QUINTIC] * 5
+
+
+def _set(shapes, seed=0, dtype=torch.bfloat16):
+    w = inputs.scaled_workload(inputs.WORKLOADS["gpt2-124m-72-matrices"], shapes)
+    Ws = [torch.from_numpy(inputs.weight_np(w, i)).cuda().to(dtype) for i in range(len(shapes))]
+    gs = [torch.from_numpy(inputs.grad_np(w, 1 + seed, i)).cuda() for i in range(len(shapes))]
+    ms = [torch.from_numpy(inputs.grad_np(w, 0, i)).cuda() for i in range(len(shapes))]
+    return Ws, gs, ms
+
+
+def _clone(ts):
+    return [t.clone() for t in ts]
+
+
+SHAPES = [(256, 128), (128, 384), (256, 128), (192, 192), (136, 200)]
+
+
+def test_bitwise_deterministic():
+    require_gpu()
+    from newton_schulz_11_b200 import api
+
+    Ws, gs, ms = _set(SHAPES)
+    W1, m1 = _clone(Ws), _clone(ms)
+    W2, m2 = _clone(Ws), _clone(ms)
+    O1 = [torch.empty_like(g) for g in gs]
+    O2 = [torch.empty_like(g) for g in gs]
+    api.muon_step(W1, gs, m1, lr=0.02, outs=O1)
+    api.muon_step(W2, gs, m2, lr=0.02, outs=O2)
+    for a, b in zip(O1 + W1 + m1, O2 + W2 + m2):
+        assert torch.equal(a, b)
+
+
+def test_waves_give_identical_results():
+    """A workspace that fits one matrix at a time gives bit-identical results."""
+    require_gpu()
+    from newton_schulz_11_b200 import api
+
+    Ws, gs, ms = _set(SHAPES)
+    W1, m1, W2, m2 = _clone(Ws), _clone(ms), _clone(Ws), _clone(ms)
+    O1 = [torch.empty_like(g) for g in gs]
+    O2 = [torch.empty_like(g) for g in gs]
+    api.muon_step(W1, gs, m1, lr=0.02, outs=O1)
+    one = max(api.workspace_size([tuple(g.shape)]) for g in gs)
+    ws = api.Workspace(gs[0].device)
+    api.muon_step(W2, gs, m2, lr=0.02, outs=O2, workspace=ws, workspace_bytes=one)
+    assert api.scratch_view([tuple(g.shape) for g in gs], len(gs) - 1, one).wave == len(gs) - 1
+    for a, b in zip(O1 + W1 + m1, O2 + W2 + m2):
+        assert torch.equal(a, b)
+
+
+def test_strided_views_match_contiguous():
+    """Parameters, grads and momentum given as column blocks of wider buffers (ld > cols)."""
+    require_gpu()
+    from newton_schulz_11_b200 import api
+
+    Ws, gs, ms = _set([(192, 128), (128, 256)], dtype=torch.float32)
+    bigW = [torch.zeros(W.shape[0], W.shape[1] + 40, device="cuda") for W in Ws]
+    bigg = [torch.zeros(g.shape[0], g.shape[1] + 24, device="cuda") for g in gs]
+    bigm = [torch.zeros(m.shape[0], m.shape[1] + 8, device="cuda") for m in ms]
+    vW = [b[:, 8: 8 + W.shape[1]] for b, W in zip(bigW, Ws)]
+    vg = [b[:, 4: 4 + g.shape[1]] for b, g in zip(bigg, gs)]
+    vm = [b[:, : m.shape[1]] for b, m in zip(bigm, ms)]
+    for v, t in zip(vW + vg + vm, Ws + gs + ms):
+        v.copy_(t)
+    Wc, mc = _clone(Ws), _clone(ms)
+    api.muon_step(Wc, gs, mc, lr=0.02, weight_decay=0.1)
+    api.muon_step(vW, vg, vm, lr=0.02, weight_decay=0.1)
+    for a, b in zip(vW + vm, Wc + mc):
+        assert torch.equal(a, b)
+    # bytes outside the views untouched
+    for b, W in zip(bigW, Ws):
+        assert torch.count_nonzero(b[:, :8]).item() == 0 and torch.count_nonzero(b[:, 8 + W.shape[1]:]).item() == 0
+
+
+def test_nan_stays_in_its_matrix():
+    require_gpu()
+    from newton_schulz_11_b200 import api
+
+    Ws, gs, ms = _set([(128, 128), (128, 256)], dtype=torch.float32)
+    gs[0][3, 5] = float("nan")
+    O = [torch.empty_like(g) for g in gs]
+    api.muon_step(Ws, gs, ms, lr=0.02, outs=O)
+    assert torch.isnan(O[0]).any()
+    assert torch.isfinite(O[1]).all() and torch.isfinite(Ws[1]).all()
+
+
+def test_checkpoint_round_trip_is_bit_identical():
+    """3 steps == 2 steps, save/load of params and momentum, 1 step."""
+    require_gpu()
+    from newton_schulz_11_b200 import api
+
+    Ws, gs, ms = _set([(256, 128), (128, 256)])
+    WA, mA = _clone(Ws), _clone(ms)
+    for _ in range(3):
+        api.muon_step(WA, gs, mA, lr=0.02, weight_decay=0.01)
+    WB, mB = _clone(Ws), _clone(ms)
+    for _ in range(2):
+        api.muon_step(WB, gs, mB, lr=0.02, weight_decay=0.01)
+    saved = [t.cpu() for t in WB + mB]
+    WC = [t.cuda() for t in saved[:2]]
+    mC = [t.cuda() for t in saved[2:]]
+    api.muon_step(WC, gs, mC, lr=0.02, weight_decay=0.01)
+    for a, b in zip(WA + mA, WC + mC):
+        assert torch.equal(a, b)
+
+
+def test_invalid_call_touches_nothing():
+    require_gpu()
+    from newton_schulz_11_b200 import api, _lib
+
+    Ws, gs, ms = _set([(64, 64)], dtype=torch.float32)
+    W0, m0 = _clone(Ws), _clone(ms)
+    with pytest.raises(_lib.MuonError):
+        api.muon_step(Ws, gs, ms, lr=0.02, beta=2.0)
+    torch.cuda.synchronize()
+    assert torch.equal(Ws[0], W0[0]) and torch.equal(ms[0], m0[0])
+
+
+def test_device_status_stays_ok():
+    require_gpu()
+    from newton_schulz_11_b200 import api, _lib
+
+    Ws, gs, ms = _set(SHAPES)
+    ws = api.Workspace(gs[0].device)
+    api.muon_step(Ws, gs, ms, lr=0.02, workspace=ws)
+    assert api.device_status(ws) == (_lib.MUON_OK, 0)
