@@ -25,8 +25,9 @@
 namespace muon {
 cudaError_t launch_momentum(const EwParams& p, cudaStream_t stream);
 cudaError_t launch_norm(const EwParams& p, cudaStream_t stream);
-cudaError_t launch_gemm(int mode, const GemmParams* p, int grid, cudaStream_t stream);
-int gemm_bn_for_mode(int mode);
+cudaError_t launch_gemm(int mode, const GemmParams* p, int max_pairs, cudaStream_t stream);
+int gemm_tile_rows();
+int gemm_tile_cols();
 }  // namespace muon
 
 namespace {
@@ -323,20 +324,17 @@ struct WaveLaunch {
   int grid_sym = 0, grid_apply = 0;
 };
 
-void fill_sym_tiles(ClassDesc& d, int64_t m, int bn) {
-  d.mb = cdiv(m, kBM);
-  d.nb = cdiv(m, bn);
-  int t = 0;
-  for (int ib = 0; ib < d.mb; ++ib) t += d.nb - (ib * kBM) / bn;
-  d.tiles_per_mat = t;
+// Symmetric products: pair tiles (I, J) with J >= I over the m x m output.
+void fill_sym_tiles(ClassDesc& d, int64_t m) {
+  d.mb = cdiv(m, gemm_tile_rows());
+  d.nb = cdiv(m, gemm_tile_cols());
+  d.tiles_per_mat = d.nb * (d.nb + 1) / 2;
   d.out_rows = d.out_cols = static_cast<int32_t>(m);
   d.i_fast = 0;
 }
 
 muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* ws, int sms, WaveLaunch* L) {
   const int nw = static_cast<int>(w.order.size());
-  const int bn_sym = gemm_bn_for_mode(kGram);
-  const int bn_apply = gemm_bn_for_mode(kApply);
   float* scale = reinterpret_cast<float*>(ws + w.off_scale);
   int32_t* status = reinterpret_cast<int32_t*>(ws);
 
@@ -356,7 +354,7 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
   base.status = status;
   int tiles_sym = 0, tiles_apply = 0;
   ClassDesc sym[kMaxClasses], app[kMaxClasses];
-  CUtensorMap map_hi[kMaxClasses][2], map_a[kMaxClasses], map_b[kMaxClasses];
+  CUtensorMap map_hi[kMaxClasses][2], map_lo[kMaxClasses], map_abuf[kMaxClasses], map_bbuf[kMaxClasses];
   for (int ci = 0; ci < static_cast<int>(w.classes.size()); ++ci) {
     const ClassPlan& c = w.classes[ci];
     const int count = static_cast<int>(c.mats.size());
@@ -367,7 +365,9 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
     __nv_bfloat16* bb = reinterpret_cast<__nv_bfloat16*>(ws + c.off_b);
     if (!encode_map(&map_hi[ci][0], hi0, count, c.rows, c.cols, c.ldx) ||
         !encode_map(&map_hi[ci][1], hi1, count, c.rows, c.cols, c.ldx) ||
-        !encode_map(&map_a[ci], ab, count, c.m, c.m, c.lda) || !encode_map(&map_b[ci], bb, count, c.m, c.m, c.lda))
+        !encode_map(&map_lo[ci], lo, count, c.rows, c.cols, c.ldx) ||
+        !encode_map(&map_abuf[ci], ab, count, c.m, c.m, c.lda) ||
+        !encode_map(&map_bbuf[ci], bb, count, c.m, c.m, c.lda))
       return MUON_ERR_CUDA;
 
     ClassDesc d{};
@@ -387,13 +387,13 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
     d.b_buf = bb;
 
     sym[ci] = d;
-    fill_sym_tiles(sym[ci], c.m, bn_sym);
+    fill_sym_tiles(sym[ci], c.m);
     sym[ci].tile_begin = tiles_sym;
     tiles_sym += count * sym[ci].tiles_per_mat;
 
     app[ci] = d;
-    app[ci].mb = cdiv(c.rows, kBM);
-    app[ci].nb = cdiv(c.cols, bn_apply);
+    app[ci].mb = cdiv(c.rows, gemm_tile_rows());
+    app[ci].nb = cdiv(c.cols, gemm_tile_cols());
     app[ci].tiles_per_mat = app[ci].mb * app[ci].nb;
     app[ci].out_rows = d.rows;
     app[ci].out_cols = d.cols;
@@ -447,17 +447,21 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
       g.cls[ci].ksize = static_cast<int32_t>(w.classes[ci].n);
       g.cls[ci].a_mn = g.cls[ci].b_mn = w.classes[ci].tall;
       g.map_a[ci] = g.map_b[ci] = map_hi[ci][cur];
+      g.map_out[ci] = map_abuf[ci];
 
       a.cls[ci] = app[ci];
       a.cls[ci].x_hi_cur = reinterpret_cast<__nv_bfloat16*>(ws + w.classes[ci].off_hi[cur]);
       a.cls[ci].x_hi_next = reinterpret_cast<__nv_bfloat16*>(ws + w.classes[ci].off_hi[cur ^ 1]);
       if (w.classes[ci].tall) {
         a.map_a[ci] = map_hi[ci][cur];
-        a.map_b[ci] = map_b[ci];
+        a.map_b[ci] = map_bbuf[ci];
       } else {
-        a.map_a[ci] = map_b[ci];
+        a.map_a[ci] = map_bbuf[ci];
         a.map_b[ci] = map_hi[ci][cur];
       }
+      a.map_in0[ci] = map_hi[ci][cur];
+      a.map_in1[ci] = map_lo[ci];
+      a.map_out[ci] = map_hi[ci][cur ^ 1];
     }
     g.total_tiles = tiles_sym;
     a.total_tiles = tiles_apply;
@@ -470,12 +474,14 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
     pp.cls[ci] = sym[ci];
     pp.cls[ci].ksize = static_cast<int32_t>(w.classes[ci].m);
     pp.cls[ci].a_mn = pp.cls[ci].b_mn = 0;
-    pp.map_a[ci] = pp.map_b[ci] = map_a[ci];
+    pp.map_a[ci] = pp.map_b[ci] = map_abuf[ci];
+    pp.map_in0[ci] = map_abuf[ci];
+    pp.map_out[ci] = map_bbuf[ci];
   }
   pp.total_tiles = tiles_sym;
   L->poly = pp;
-  L->grid_sym = std::max(1, std::min(tiles_sym, sms));
-  L->grid_apply = std::max(1, std::min(tiles_apply, sms));
+  L->grid_sym = std::max(1, sms / 2);   // CTA pairs available
+  L->grid_apply = std::max(1, sms / 2);
   return MUON_OK;
 }
 

@@ -32,6 +32,8 @@ enum WaitSite : int {
   kSiteEpilogueFull = 4,
   kSiteTeardownTma = 5,
   kSiteTeardownMma = 6,
+  kSiteEpilogueIn = 7,
+  kSiteProducerEpi = 8,
 };
 
 // One shape class of a wave: `count` matrices of the same rows x cols, stored
@@ -74,6 +76,9 @@ struct UpdMat {
 struct GemmParams {
   CUtensorMap map_a[kMaxClasses];   // operand A of the launch, per class
   CUtensorMap map_b[kMaxClasses];   // operand B
+  CUtensorMap map_in0[kMaxClasses];  // epilogue input: apply -> hi of X, polynomial -> A
+  CUtensorMap map_in1[kMaxClasses];  // epilogue input: apply -> lo of X (written back in place)
+  CUtensorMap map_out[kMaxClasses];  // epilogue output: Gram -> A, polynomial -> B, apply -> next hi
   ClassDesc cls[kMaxClasses];
   int32_t num_classes;
   int32_t total_tiles;
