@@ -48,6 +48,8 @@ __device__ __forceinline__ float ew_one(float g, float& m, float beta, int neste
 
 __global__ void __launch_bounds__(kEwThreads) muon_momentum_kernel(const __grid_constant__ EwParams p) {
   __shared__ float red[kEwThreads / 32];
+  griddep_launch_dependents();
+  griddep_wait();  // the previous step may still read the hi/lo buffers this writes
   const int chunk = blockIdx.x;
   const int i = find_matrix(p, chunk);
   const EwMat& t = p.mats[i];
@@ -113,6 +115,8 @@ __global__ void __launch_bounds__(kEwThreads) muon_momentum_kernel(const __grid_
 // fixed order.
 __global__ void __launch_bounds__(kEwThreads) muon_norm_kernel(const __grid_constant__ EwParams p) {
   __shared__ double red[kEwThreads];
+  griddep_launch_dependents();
+  griddep_wait();
   const EwMat& t = p.mats[blockIdx.x];
   double s = 0.0;
   for (int k = threadIdx.x; k < t.nchunks; k += kEwThreads) s += static_cast<double>(p.partials[t.chunk_begin + k]);
@@ -129,14 +133,24 @@ __global__ void __launch_bounds__(kEwThreads) muon_norm_kernel(const __grid_cons
   }
 }
 
-cudaError_t launch_momentum(const EwParams& p, cudaStream_t stream) {
-  muon_momentum_kernel<<<p.total_chunks, kEwThreads, 0, stream>>>(p);
-  return cudaGetLastError();
+template <typename K>
+static cudaError_t launch_pdl(K kernel, int grid, const EwParams& p, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kEwThreads, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
-cudaError_t launch_norm(const EwParams& p, cudaStream_t stream) {
-  muon_norm_kernel<<<p.n, kEwThreads, 0, stream>>>(p);
-  return cudaGetLastError();
+cudaError_t launch_momentum(const EwParams& p, cudaStream_t stream) {
+  return launch_pdl(muon_momentum_kernel, p.total_chunks, p, stream);
 }
+
+cudaError_t launch_norm(const EwParams& p, cudaStream_t stream) { return launch_pdl(muon_norm_kernel, p.n, p, stream); }
 
 }  // namespace muon

@@ -41,6 +41,7 @@ constexpr size_t kHeaderBytes = 256;
 constexpr size_t kBufAlign = 1024;
 constexpr int64_t kChunkElems = 16384;
 constexpr int64_t kMaxSide = int64_t(1) << 24;
+constexpr int kStagedApplyMaxM = 1024;  // Gram side up to which the apply stages hi/lo by TMA
 
 std::atomic<long long> g_timeout_us{2000000};
 
@@ -92,15 +93,16 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 3-D bf16 map over `count` matrices of rows x cols (row stride ld elements), 64x64 boxes,
-// 128-byte swizzle, zero fill outside the matrix.
-bool encode_map(CUtensorMap* map, void* base, int64_t count, int64_t rows, int64_t cols, int64_t ld) {
+// 3-D bf16 map over `count` matrices of rows x cols (row stride ld elements), boxes of
+// 64 columns x box_rows rows, 128-byte swizzle, zero fill outside the matrix.
+bool encode_map(CUtensorMap* map, void* base, int64_t count, int64_t rows, int64_t cols, int64_t ld,
+                uint32_t box_rows) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(count)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld * 2), static_cast<cuuint64_t>(ld * rows * 2)};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(kBox), static_cast<cuuint32_t>(kBox), 1};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(kBox), box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -354,7 +356,9 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
   base.status = status;
   int tiles_sym = 0, tiles_apply = 0;
   ClassDesc sym[kMaxClasses], app[kMaxClasses];
-  CUtensorMap map_hi[kMaxClasses][2], map_lo[kMaxClasses], map_abuf[kMaxClasses], map_bbuf[kMaxClasses];
+  // operand maps: 64 x 128 boxes; epilogue store maps: 64 x 64 boxes
+  CUtensorMap op_hi[kMaxClasses][2], op_a[kMaxClasses], op_b[kMaxClasses];
+  CUtensorMap st_hi[kMaxClasses][2], st_lo[kMaxClasses], st_a[kMaxClasses], st_b[kMaxClasses];
   for (int ci = 0; ci < static_cast<int>(w.classes.size()); ++ci) {
     const ClassPlan& c = w.classes[ci];
     const int count = static_cast<int>(c.mats.size());
@@ -363,11 +367,15 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
     __nv_bfloat16* lo = reinterpret_cast<__nv_bfloat16*>(ws + c.off_lo);
     __nv_bfloat16* ab = reinterpret_cast<__nv_bfloat16*>(ws + c.off_a);
     __nv_bfloat16* bb = reinterpret_cast<__nv_bfloat16*>(ws + c.off_b);
-    if (!encode_map(&map_hi[ci][0], hi0, count, c.rows, c.cols, c.ldx) ||
-        !encode_map(&map_hi[ci][1], hi1, count, c.rows, c.cols, c.ldx) ||
-        !encode_map(&map_lo[ci], lo, count, c.rows, c.cols, c.ldx) ||
-        !encode_map(&map_abuf[ci], ab, count, c.m, c.m, c.lda) ||
-        !encode_map(&map_bbuf[ci], bb, count, c.m, c.m, c.lda))
+    if (!encode_map(&op_hi[ci][0], hi0, count, c.rows, c.cols, c.ldx, 128) ||
+        !encode_map(&op_hi[ci][1], hi1, count, c.rows, c.cols, c.ldx, 128) ||
+        !encode_map(&op_a[ci], ab, count, c.m, c.m, c.lda, 128) ||
+        !encode_map(&op_b[ci], bb, count, c.m, c.m, c.lda, 128) ||
+        !encode_map(&st_hi[ci][0], hi0, count, c.rows, c.cols, c.ldx, 64) ||
+        !encode_map(&st_hi[ci][1], hi1, count, c.rows, c.cols, c.ldx, 64) ||
+        !encode_map(&st_lo[ci], lo, count, c.rows, c.cols, c.ldx, 64) ||
+        !encode_map(&st_a[ci], ab, count, c.m, c.m, c.lda, 64) ||
+        !encode_map(&st_b[ci], bb, count, c.m, c.m, c.lda, 64))
       return MUON_ERR_CUDA;
 
     ClassDesc d{};
@@ -439,29 +447,56 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
     }
   }
 
+  // Classes with the longest reductions (the most expensive tiles) go first, so the
+  // round-robin tile assignment balances the pairs' work.
+  const int nc = base.num_classes;
+  std::vector<int> ord_sym(nc), ord_app(nc);
+  for (int i = 0; i < nc; ++i) ord_sym[i] = ord_app[i] = i;
+  std::stable_sort(ord_sym.begin(), ord_sym.end(),
+                   [&](int x, int y) { return w.classes[x].n > w.classes[y].n; });
+  std::stable_sort(ord_app.begin(), ord_app.end(),
+                   [&](int x, int y) { return w.classes[x].m > w.classes[y].m; });
+  tiles_sym = tiles_apply = 0;
+  for (int k = 0; k < nc; ++k) {
+    sym[ord_sym[k]].tile_begin = tiles_sym;
+    tiles_sym += sym[ord_sym[k]].count * sym[ord_sym[k]].tiles_per_mat;
+    app[ord_app[k]].tile_begin = tiles_apply;
+    tiles_apply += app[ord_app[k]].count * app[ord_app[k]].tiles_per_mat;
+  }
+  // The apply runs the staged variant while every Gram side is short: its tiles then
+  // have short reductions, and moving the epilogue's hi/lo by TMA matters more than the
+  // main loop's k-block depth.
+  int max_m = 0;
+  for (const ClassPlan& c : w.classes) max_m = std::max(max_m, static_cast<int>(c.m));
+  const bool staged = max_m <= kStagedApplyMaxM;
   for (int cur = 0; cur < 2; ++cur) {
     GemmParams g = base;
     GemmParams a = base;
-    for (int ci = 0; ci < base.num_classes; ++ci) {
-      g.cls[ci] = sym[ci];
-      g.cls[ci].ksize = static_cast<int32_t>(w.classes[ci].n);
-      g.cls[ci].a_mn = g.cls[ci].b_mn = w.classes[ci].tall;
-      g.map_a[ci] = g.map_b[ci] = map_hi[ci][cur];
-      g.map_out[ci] = map_abuf[ci];
+    a.staged = staged ? 1 : 0;
+    for (int k = 0; k < nc; ++k) {
+      const int ci = ord_sym[k];
+      g.cls[k] = sym[ci];
+      g.cls[k].ksize = static_cast<int32_t>(w.classes[ci].n);
+      g.cls[k].a_mn = g.cls[k].b_mn = w.classes[ci].tall;
+      g.map_a[k] = g.map_b[k] = op_hi[ci][cur];
+      g.map_out[k] = st_a[ci];
 
-      a.cls[ci] = app[ci];
-      a.cls[ci].x_hi_cur = reinterpret_cast<__nv_bfloat16*>(ws + w.classes[ci].off_hi[cur]);
-      a.cls[ci].x_hi_next = reinterpret_cast<__nv_bfloat16*>(ws + w.classes[ci].off_hi[cur ^ 1]);
-      if (w.classes[ci].tall) {
-        a.map_a[ci] = map_hi[ci][cur];
-        a.map_b[ci] = map_bbuf[ci];
+      const int cj = ord_app[k];
+      a.cls[k] = app[cj];
+      a.cls[k].x_hi_cur = reinterpret_cast<__nv_bfloat16*>(ws + w.classes[cj].off_hi[cur]);
+      a.cls[k].x_hi_next = reinterpret_cast<__nv_bfloat16*>(ws + w.classes[cj].off_hi[cur ^ 1]);
+      const CUtensorMap& x_op = staged ? st_hi[cj][cur] : op_hi[cj][cur];
+      const CUtensorMap& b_op = staged ? st_b[cj] : op_b[cj];
+      if (w.classes[cj].tall) {
+        a.map_a[k] = x_op;
+        a.map_b[k] = b_op;
       } else {
-        a.map_a[ci] = map_bbuf[ci];
-        a.map_b[ci] = map_hi[ci][cur];
+        a.map_a[k] = b_op;
+        a.map_b[k] = x_op;
       }
-      a.map_in0[ci] = map_hi[ci][cur];
-      a.map_in1[ci] = map_lo[ci];
-      a.map_out[ci] = map_hi[ci][cur ^ 1];
+      a.map_in[k] = st_hi[cj][cur];
+      a.map_out[k] = st_hi[cj][cur ^ 1];
+      a.map_out2[k] = st_lo[cj];
     }
     g.total_tiles = tiles_sym;
     a.total_tiles = tiles_apply;
@@ -470,13 +505,20 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
     static_cast<GemmParams&>(L->fin[cur]) = a;
   }
   GemmParams pp = base;
-  for (int ci = 0; ci < base.num_classes; ++ci) {
-    pp.cls[ci] = sym[ci];
-    pp.cls[ci].ksize = static_cast<int32_t>(w.classes[ci].m);
-    pp.cls[ci].a_mn = pp.cls[ci].b_mn = 0;
-    pp.map_a[ci] = pp.map_b[ci] = map_abuf[ci];
-    pp.map_in0[ci] = map_abuf[ci];
-    pp.map_out[ci] = map_bbuf[ci];
+  for (int k = 0; k < nc; ++k) {
+    const int ci = ord_app[k];  // the polynomial's reduction is m, like the apply's
+    pp.cls[k] = sym[ci];
+    pp.cls[k].ksize = static_cast<int32_t>(w.classes[ci].m);
+    pp.cls[k].a_mn = pp.cls[k].b_mn = 0;
+    pp.map_a[k] = pp.map_b[k] = op_a[ci];
+    pp.map_out[k] = st_b[ci];
+  }
+  {
+    int tb = 0;
+    for (int k = 0; k < nc; ++k) {
+      pp.cls[k].tile_begin = tb;
+      tb += pp.cls[k].count * pp.cls[k].tiles_per_mat;
+    }
   }
   pp.total_tiles = tiles_sym;
   L->poly = pp;

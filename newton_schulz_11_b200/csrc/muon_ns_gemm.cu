@@ -47,20 +47,30 @@
 
 namespace muon {
 
-template <int MODE>
+// Two variants share the kernel.  Streamed (SMALL = false, every mode): 128-deep k-blocks,
+// three 64 KB stages per CTA, a 32 KB epilogue staging area; epilogue inputs are read
+// from global memory.  Staged (SMALL = true, apply modes when the Gram side m is at most
+// 1024): 64-deep k-blocks, three 32 KB stages, and the tile's hi/lo inputs (128 KB per CTA)
+// loaded by TMA into shared memory -- the apply is bound by HBM traffic there, and TMA
+// moves it in full lines.
+template <int MODE, bool SMALL = false>
 struct Lay {
   static constexpr bool kSym = MODE == kGram || MODE == kPoly;
+  static_assert(!(SMALL && kSym), "the staged variant is an apply");
   static constexpr int TM = 256;  // pair tile rows (128 per CTA)
   static constexpr int TN = 256;  // pair tile columns = UMMA N
-  static constexpr int S = MODE == kGram ? 5 : 3;
+  static constexpr int BK = SMALL ? 64 : 128;
+  static constexpr int S = 3;
   static constexpr int NEPI = 8;
-  static constexpr int kABytes = kBM * kBK * 2;  // this CTA's 128 rows of A
-  static constexpr int kBBytes = kBM * kBK * 2;  // this CTA's 128 rows (half of N) of B
+  static constexpr int kBox64 = 64 * 64 * 2;       // one 64 x 64 box: 8 KB
+  static constexpr int kHalf = kBM * kBox * 2;      // one 64 x 128 box: 16 KB
+  static constexpr int kABytes = kBM * BK * 2;      // this CTA's 128 rows x BK of A
+  static constexpr int kBBytes = kBM * BK * 2;      // this CTA's 128 rows (half of N) x BK of B
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kRing = S * kStageBytes;
-  static constexpr int kBlk = kBM * 128 * 2;  // one staged 128 x 128 bf16 block
-  // Gram: D, T.  Polynomial: D, T, Ain (128 x 256).  Apply: hi, lo (128 x 256 each).
-  static constexpr int kEpi = MODE == kGram ? 2 * kBlk : 4 * kBlk;
+  // streamed: one 64-column quarter of this CTA's 128 x 256 tile at a time (symmetric
+  // modes D_q and T_q, apply hi_q and lo_q); staged: the tile's hi and lo, 128 x 256 each
+  static constexpr int kEpi = SMALL ? 8 * kHalf : 2 * kHalf;
   static constexpr int kBarOff = kRing + kEpi;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;
   static constexpr int kEpiThreads = 32 * NEPI;
@@ -133,54 +143,82 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t) {
   return r;
 }
 
-// One 64-row (K-major) or 64-column (MN-major) slab of an operand tile, completing on
-// the leader CTA's mbarrier.
-__device__ __forceinline__ void load_box_pair(void* dst, const CUtensorMap* map, int mn_major, int mn0, int k0,
-                                              int mat, uint32_t bar_cluster) {
+// Half i of an operand tile (128 MN x BK), completing on the leader CTA's mbarrier.
+//   BK = 128 (64 x 128 boxes): K-major -> K columns [k0 + 64 i, +64) of 128 rows;
+//                              MN-major -> MN columns [mn0 + 64 i, +64) of 128 K-rows.
+//   BK = 64 (64 x 64 boxes):   K-major -> rows [mn0 + 64 i, +64) of 64 K columns;
+//                              MN-major -> MN columns [mn0 + 64 i, +64) of 64 K-rows.
+// In both cases half i lands at i x (its bytes), which is the layout operand_desc reads.
+template <int BK>
+__device__ __forceinline__ void load_half_pair(void* dst, const CUtensorMap* map, int mn_major, int mn0, int k0,
+                                               int i, int mat, uint32_t bar_cluster) {
   if (mn_major)
-    tma_load_3d_pair(dst, map, bar_cluster, mn0, k0, mat);
+    tma_load_3d_pair(dst, map, bar_cluster, mn0 + 64 * i, k0, mat);
+  else if (BK == 128)
+    tma_load_3d_pair(dst, map, bar_cluster, k0 + 64 * i, mn0, mat);
   else
-    tma_load_3d_pair(dst, map, bar_cluster, k0, mn0, mat);
+    tma_load_3d_pair(dst, map, bar_cluster, k0, mn0 + 64 * i, mat);
 }
 
+// Shared-memory descriptor of the kk-th 16-deep K slice (kk < BK / 16) of a staged operand:
+//   K-major : 128 rows x 128 B per 64-deep K half (16 KB); slice kk in half kk / 4, 32 B per
+//             slice; 8-row groups 1 KB apart (SBO).
+//   MN-major: two halves (64 MN each) of BK K-rows x 128 B; slice kk starts at K-row 16 kk
+//             (2 KB per slice); 8-row groups 1 KB apart (SBO), halves BK x 128 B apart (LBO).
+template <int BK>
 __device__ __forceinline__ uint64_t operand_desc(uint32_t tile_addr, int mn_major, int kk) {
-  return mn_major ? smem_desc_sw128(tile_addr + kk * 2048u, 8192u, 1024u)
-                  : smem_desc_sw128(tile_addr + kk * 32u, 16u, 1024u);
+  return mn_major ? smem_desc_sw128(tile_addr + kk * 2048u, BK * 128u, 1024u)
+                  : smem_desc_sw128(tile_addr + (kk >> 2) * 16384u + (kk & 3) * 32u, 16u, 1024u);
 }
 
 // ------------------------------------------------------------------ staging layouts
 //
-// A staged region of 128 rows x (64 NCB) columns of bf16 is a grid of 64 x 64 boxes with
-// 128-byte swizzle, as TMA reads and writes them: box (rb, cb) at (rb NCB + cb) * 8 KB,
-// row rr of a box at rr * 128 B, and its 16-byte chunk k at chunk k ^ (rr & 7).  Eight
-// consecutive rows then hit eight different bank groups: conflict-free row access.
-template <int NCB>
-__device__ __forceinline__ uint32_t chunk_off(int r, int c16) {
+// Epilogue staging, as TMA stores read it (64 x 64 boxes, 128-byte swizzle: row rr of a box at
+// rr * 128 B, its 16-byte chunk k at chunk k ^ (rr & 7)):
+//   Q (offset 0)     128 rows x 64 columns: D_q, or the new hi of the apply
+//   T (offset 16 KB) symmetric modes: 64 rows x 128 columns (the transpose of D_q), as two
+//                    boxes side by side; apply: 128 x 64, the new lo, laid out like Q
+// Eight consecutive rows hit eight different bank groups: row-wise access is conflict-free.
+__device__ __forceinline__ uint32_t q_chunk(int r, int c16) { return static_cast<uint32_t>(r * 128 + ((c16 ^ (r & 7)) << 4)); }
+
+// Staged apply: the tile's hi (and lo) as 128 rows x 256 columns, a 2 x 4 grid of 64 x 64
+// boxes in the same swizzle: box (rb, cb) at (4 rb + cb) x 8 KB.
+__device__ __forceinline__ uint32_t region_chunk(int r, int c16) {
   const int rr = r & 63;
-  return static_cast<uint32_t>((((r >> 6) * NCB + (c16 >> 3)) << 13) + rr * 128 + (((c16 & 7) ^ (rr & 7)) << 4));
+  return static_cast<uint32_t>((((r >> 6) * 4 + (c16 >> 3)) << 13) + rr * 128 + (((c16 & 7) ^ (rr & 7)) << 4));
 }
 
-template <int NCB>
-__device__ __forceinline__ uint32_t elem_off(int r, int c) {
-  return chunk_off<NCB>(r, c >> 3) + ((c & 7) << 1);
+// TMA transfers of the staged region's column boxes [cb0, cb0 + ncb) at rows row0..,
+// columns col0.. of matrix `mat`.  Parts outside the matrix are read as zero and not written.
+__device__ __forceinline__ void store_region(const CUtensorMap* map, const uint8_t* buf, int cb0, int ncb, int row0,
+                                             int col0, int mat) {
+#pragma unroll 1
+  for (int rb = 0; rb < 2; ++rb)
+#pragma unroll 1
+    for (int cb = cb0; cb < cb0 + ncb; ++cb)
+      tma_store_3d(map, buf + ((4 * rb + cb) << 13), col0 + 64 * cb, row0 + 64 * rb, mat);
 }
 
-__device__ __forceinline__ void unpack8(uint4 w, float* f) {
-  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+__device__ __forceinline__ void load_region(uint8_t* buf, const CUtensorMap* map, uint64_t* bar, int row0, int col0,
+                                            int mat) {
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    f[2 * e] = bf16_bits_to_float(ws[e] & 0xFFFFu);
-    f[2 * e + 1] = bf16_bits_to_float(ws[e] >> 16);
-  }
+  for (int rb = 0; rb < 2; ++rb)
+#pragma unroll
+    for (int cb = 0; cb < 4; ++cb)
+      tma_load_3d(buf + ((4 * rb + cb) << 13), map, bar, col0 + 64 * cb, row0 + 64 * rb, mat);
 }
 
 __device__ __forceinline__ uint4 pack8(const uint32_t* b) {
   return make_uint4(b[0] | (b[1] << 16), b[2] | (b[3] << 16), b[4] | (b[5] << 16), b[6] | (b[7] << 16));
 }
 
-__device__ __forceinline__ void st_u16(uint8_t* base, uint32_t off, uint32_t bits) {
-  *reinterpret_cast<unsigned short*>(base + off) = static_cast<unsigned short>(bits);
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
 }
+
+__device__ __forceinline__ float lo_bf16(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float hi_bf16(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 __device__ __forceinline__ float bf16_at(const __nv_bfloat16* p) {
   return bf16_bits_to_float(__bfloat16_as_ushort(*p));
@@ -190,172 +228,231 @@ __device__ __forceinline__ void put_bf16(__nv_bfloat16* p, uint32_t bits) {
   *p = __ushort_as_bfloat16(static_cast<unsigned short>(bits));
 }
 
-// Stores / loads a staged region of 128 rows x 64 NCB columns at rows row0.., columns
-// col0.. of matrix `mat`; parts outside the matrix are not written / read as zero.
-template <int NCB>
-__device__ __forceinline__ void store_region(const CUtensorMap* map, const uint8_t* buf, int cb0, int ncb, int row0,
-                                             int col0, int mat) {
-#pragma unroll 1
-  for (int rb = 0; rb < 2; ++rb)
-#pragma unroll 1
-    for (int cb = cb0; cb < cb0 + ncb; ++cb)
-      tma_store_3d(map, buf + ((rb * NCB + cb) << 13), col0 + 64 * cb, row0 + 64 * rb, mat);
+// 32 consecutive bf16 of one row (four 16-byte loads), zero past `valid` columns or when
+// `live` is false.  `row` is 16-byte aligned; `valid` columns exist in its padded extent.
+__device__ __forceinline__ void load_row32(const __nv_bfloat16* row, int valid, bool live, uint4 (&w)[4]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (live && 8 * q < valid)
+      w[q] = __ldg(reinterpret_cast<const uint4*>(row) + q);
+    else
+      w[q] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  if (live && valid < 32 && valid > 0) {  // ragged tail inside the last loaded chunk
+    uint32_t* e = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (2 * j >= valid) e[j] = 0u;
+      else if (2 * j + 1 >= valid) e[j] &= 0xFFFFu;
+    }
+  }
 }
 
-template <int NCB>
-__device__ __forceinline__ void load_region(uint8_t* buf, const CUtensorMap* map, uint64_t* bar, int row0, int col0,
-                                            int mat) {
-#pragma unroll
-  for (int rb = 0; rb < 2; ++rb)
-#pragma unroll
-    for (int cb = 0; cb < NCB; ++cb)
-      tma_load_3d(buf + ((rb * NCB + cb) << 13), map, bar, col0 + 64 * cb, row0 + 64 * rb, mat);
+// Stores 128 x 64 staged at Q (two boxes) at rows row0.., columns col0..
+__device__ __forceinline__ void store_q(const CUtensorMap* map, const uint8_t* q, int row0, int col0, int mat) {
+  tma_store_3d(map, q, col0, row0, mat);
+  tma_store_3d(map, q + 8192, col0, row0 + 64, mat);
+}
+
+// Stores 64 x 128 staged at T (two boxes side by side) at rows row0.., columns col0..
+__device__ __forceinline__ void store_t(const CUtensorMap* map, const uint8_t* t, int row0, int col0, int mat) {
+  tma_store_3d(map, t, col0, row0, mat);
+  tma_store_3d(map, t + 8192, col0 + 64, row0, mat);
 }
 
 // ------------------------------------------------------------------ epilogues
 
-// One 128 x 128 block of a symmetric product: block row r of this CTA, the 64 columns
-// [64 h, 64 h + 64) of the block; the block's accumulator columns start at 128 hh.
-// Off-diagonal: the row goes to D, its transpose to T.  Diagonal: D gets the upper
-// triangle from the row owners and the lower triangle mirrored from it.
+// One 64-column quarter of a symmetric product.  The thread owns row r of this CTA's
+// 128-row block and the quarter's columns [32 h, 32 h + 32), whose accumulators start at
+// TMEM column tcol.  Off-diagonal block: the row goes to Q and its transpose to T.
+// Diagonal block: the whole block goes to Q; the MMA forms (r, c) and (c, r) from the
+// same products in the same order, so it is symmetric as computed.
 template <int MODE>
-__device__ __forceinline__ void sym_block(const GemmParams& p, float mul, bool diag, int r, int h, int hh,
-                                          uint32_t tacc, uint8_t* D, uint8_t* T, const uint8_t* Ain) {
-#pragma unroll 1
-  for (int k = 0; k < 2; ++k) {
-    const int c0 = 64 * h + 32 * k;
-    uint32_t v[32];
-    tmem_ld_32x32b_x32(tacc + 128 * hh + c0, v);
-    float f[32];
-    if (MODE == kPoly) {
+__device__ __forceinline__ void sym_quarter(const GemmParams& p, float mul, bool diag, int r, int h, uint32_t tcol,
+                                            uint8_t* Q, uint8_t* T, const uint4 (&ain)[4]) {
+  uint32_t v[32];
+  tmem_ld_32x32b_x32(tcol, v);
+  tmem_wait_ld();
+  const uint32_t* a = reinterpret_cast<const uint32_t*>(ain);
+  uint32_t pk[16];
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        unpack8(*reinterpret_cast<const uint4*>(Ain + chunk_off<4>(r, ((128 * hh + c0) >> 3) + q)), f + 8 * q);
+  for (int i = 0; i < 16; ++i) {
+    float x0 = __uint_as_float(v[2 * i]), x1 = __uint_as_float(v[2 * i + 1]);
+    if (MODE == kPoly) {
+      x0 = fmaf(p.c, x0, p.b * lo_bf16(a[i]));
+      x1 = fmaf(p.c, x1, p.b * hi_bf16(a[i]));
+    } else {
+      x0 *= mul;
+      x1 *= mul;
     }
-    tmem_wait_ld();
-    uint32_t bits[32];
+    pk[i] = pack_bf16x2(x0, x1);
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    *reinterpret_cast<uint4*>(Q + q_chunk(r, 4 * h + k)) = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+  if (!diag) {
+    // T[c][r], c = 32 h + j: box r / 64, row c, 16-byte chunk ((r & 63) / 8) ^ (c & 7)
+    uint8_t* tb = T + ((r >> 6) << 13) + ((r & 7) << 1) + (32 * h) * 128;
+    const int rch = (r & 63) >> 3;
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
-      const float acc = __uint_as_float(v[j]);
-      bits[j] = float_to_bf16_bits(MODE == kPoly ? fmaf(p.c, acc, p.b * f[j]) : acc * mul);
+      const uint32_t bits = (j & 1) ? (pk[j >> 1] >> 16) : (pk[j >> 1] & 0xFFFFu);
+      *reinterpret_cast<unsigned short*>(tb + j * 128 + ((rch ^ (j & 7)) << 4)) = static_cast<unsigned short>(bits);
     }
-    if (!diag) {
+  }
+}
+
+// Final epilogue for 32 columns of one row: x holds the orthogonalised update for tile
+// columns [c0, c0 + 32) of this CTA's tile row r;  O <- x  and/or  W <- W decay - lr_scale x.
+template <int MODE>
+__device__ __forceinline__ void write_update(const FinalParams& p, const ClassDesc& cd, const Tile& tl, int rank,
+                                             int r, int c0, const float (&x)[32]) {
+  const int R = Lay<MODE>::TM * tl.I + kBM * rank + r;
+  const int C0 = Lay<MODE>::TN * tl.J + c0;
+  const int cols = cd.cols;
+  if (R >= cd.rows || C0 >= cols) return;
+  const bool full = C0 + 32 <= cols;
+  const UpdMat& u = p.upd[cd.mat_base + tl.mat];
+  if (u.out != nullptr) {
+    float* o = u.out + static_cast<int64_t>(R) * cols + C0;
+    if (full && u.vec_out) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4*>(D + chunk_off<2>(r, (c0 >> 3) + q)) = pack8(bits + 8 * q);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) st_u16(T, elem_off<2>(c0 + j, r), bits[j]);
+      for (int q = 0; q < 8; ++q)
+        reinterpret_cast<float4*>(o)[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
     } else {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int c = c0 + j;
-        if (c >= r) st_u16(D, elem_off<2>(r, c), bits[j]);
-        if (c > r) st_u16(D, elem_off<2>(c, r), bits[j]);
+      for (int j = 0; j < 32; ++j)
+        if (C0 + j < cols) o[j] = x[j];
+    }
+  }
+  if (u.param != nullptr) {
+    const float decay = p.decay, ls = u.lr_scale;
+    if (u.param_bf16) {
+      __nv_bfloat16* w = static_cast<__nv_bfloat16*>(u.param) + static_cast<int64_t>(R) * u.ld_param + C0;
+      if (full && u.vec_param) {
+        uint4 raw[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) raw[q] = reinterpret_cast<const uint4*>(w)[q];
+        const uint32_t* rw = reinterpret_cast<const uint32_t*>(raw);
+        uint32_t wb[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          wb[i] = pack_bf16x2(fmaf(-ls, x[2 * i], lo_bf16(rw[i]) * decay), fmaf(-ls, x[2 * i + 1], hi_bf16(rw[i]) * decay));
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          reinterpret_cast<uint4*>(w)[q] = make_uint4(wb[4 * q], wb[4 * q + 1], wb[4 * q + 2], wb[4 * q + 3]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (C0 + j < cols) put_bf16(w + j, float_to_bf16_bits(fmaf(-ls, x[j], bf16_at(w + j) * decay)));
+      }
+    } else {
+      float* w = static_cast<float*>(u.param) + static_cast<int64_t>(R) * u.ld_param + C0;
+      if (full && u.vec_param) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          float4 t = reinterpret_cast<float4*>(w)[q];
+          t.x = fmaf(-ls, x[4 * q], t.x * decay);
+          t.y = fmaf(-ls, x[4 * q + 1], t.y * decay);
+          t.z = fmaf(-ls, x[4 * q + 2], t.z * decay);
+          t.w = fmaf(-ls, x[4 * q + 3], t.w * decay);
+          reinterpret_cast<float4*>(w)[q] = t;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (C0 + j < cols) w[j] = fmaf(-ls, x[j], w[j] * decay);
       }
     }
   }
 }
 
-// X update for the 32 tile columns [c0, c0 + 32) of this CTA's tile row r:
-// x = s (a (hi + lo) + acc), hi/lo read from the staged 128 x 256 input region.  kApply
-// writes the new hi/lo pair back in place; kApplyLast updates W and/or writes O.
+// X update for the 32 tile columns [c0, c0 + 32) of this CTA's tile row r, with the old
+// hi/lo pair already in registers: x = s (a (hi + lo) + acc).  kApply returns the new
+// pair packed (hb, lb); kApplyLast updates W and/or writes O in global memory.
 template <int MODE>
-__device__ __forceinline__ void apply_cols(const typename ParamsOf<MODE>::type& p, const ClassDesc& cd,
-                                           const Tile& tl, int rank, int r, int c0, uint32_t tacc, uint8_t* hib,
-                                           uint8_t* lob, float s) {
+__device__ __forceinline__ void apply_quarter(const typename ParamsOf<MODE>::type& p, const ClassDesc& cd,
+                                              const Tile& tl, int rank, int r, int c0, uint32_t tcol,
+                                              const uint4 (&xh4)[4], const uint4 (&xl4)[4], float s,
+                                              uint32_t (&hb)[16], uint32_t (&lb)[16]) {
   uint32_t v[32];
-  tmem_ld_32x32b_x32(tacc + c0, v);
-  float xh[32], xl[32];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint32_t o = chunk_off<4>(r, (c0 >> 3) + q);
-    unpack8(*reinterpret_cast<const uint4*>(hib + o), xh + 8 * q);
-    unpack8(*reinterpret_cast<const uint4*>(lob + o), xl + 8 * q);
-  }
+  tmem_ld_32x32b_x32(tcol, v);
   tmem_wait_ld();
+  const uint32_t* xh = reinterpret_cast<const uint32_t*>(xh4);
+  const uint32_t* xl = reinterpret_cast<const uint32_t*>(xl4);
   float x[32];
 #pragma unroll
-  for (int j = 0; j < 32; ++j) x[j] = s * fmaf(p.a, xh[j] + xl[j], __uint_as_float(v[j]));
+  for (int i = 0; i < 16; ++i) {
+    x[2 * i] = s * fmaf(p.a, lo_bf16(xh[i]) + lo_bf16(xl[i]), __uint_as_float(v[2 * i]));
+    x[2 * i + 1] = s * fmaf(p.a, hi_bf16(xh[i]) + hi_bf16(xl[i]), __uint_as_float(v[2 * i + 1]));
+  }
   if constexpr (MODE == kApply) {
-    uint32_t hb[32], lb[32];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) split_hi_lo(x[j], hb[j], lb[j]);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint32_t o = chunk_off<4>(r, (c0 >> 3) + q);
-      *reinterpret_cast<uint4*>(hib + o) = pack8(hb + 8 * q);
-      *reinterpret_cast<uint4*>(lob + o) = pack8(lb + 8 * q);
+    for (int i = 0; i < 16; ++i) {
+      uint32_t h0, l0, h1, l1;
+      split_hi_lo(x[2 * i], h0, l0);
+      split_hi_lo(x[2 * i + 1], h1, l1);
+      hb[i] = h0 | (h1 << 16);
+      lb[i] = l0 | (l1 << 16);
     }
   } else {
-    const int R = Lay<MODE>::TM * tl.I + kBM * rank + r;
-    const int C0 = Lay<MODE>::TN * tl.J + c0;
-    const int cols = cd.cols;
-    if (R >= cd.rows || C0 >= cols) return;
-    const bool full = C0 + 32 <= cols;
-    const UpdMat& u = p.upd[cd.mat_base + tl.mat];
-    if (u.out != nullptr) {
-      float* o = u.out + static_cast<int64_t>(R) * cols + C0;
-      if (full && u.vec_out) {
+    (void)hb;
+    (void)lb;
+    write_update<MODE>(p, cd, tl, rank, r, c0, x);
+  }
+}
+
+// Staged variant of the same update: the old pair is read from the staged region, and
+// kApply writes the new pair back in place (the region is then stored by TMA).
+template <int MODE>
+__device__ __forceinline__ void apply_staged(const typename ParamsOf<MODE>::type& p, const ClassDesc& cd,
+                                             const Tile& tl, int rank, int r, int c0, uint32_t tcol, uint8_t* hib,
+                                             uint8_t* lob, float s) {
+  uint32_t v[32];
+  tmem_ld_32x32b_x32(tcol, v);
+  uint4 xh4[4], xl4[4];
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          reinterpret_cast<float4*>(o)[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
-      } else {
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t o = region_chunk(r, (c0 >> 3) + q);
+    xh4[q] = *reinterpret_cast<const uint4*>(hib + o);
+    xl4[q] = *reinterpret_cast<const uint4*>(lob + o);
+  }
+  tmem_wait_ld();
+  const uint32_t* xh = reinterpret_cast<const uint32_t*>(xh4);
+  const uint32_t* xl = reinterpret_cast<const uint32_t*>(xl4);
+  float x[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (C0 + j < cols) o[j] = x[j];
-      }
+  for (int i = 0; i < 16; ++i) {
+    x[2 * i] = s * fmaf(p.a, lo_bf16(xh[i]) + lo_bf16(xl[i]), __uint_as_float(v[2 * i]));
+    x[2 * i + 1] = s * fmaf(p.a, hi_bf16(xh[i]) + hi_bf16(xl[i]), __uint_as_float(v[2 * i + 1]));
+  }
+  if constexpr (MODE == kApply) {
+    uint32_t hb[16], lb[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      uint32_t h0, l0, h1, l1;
+      split_hi_lo(x[2 * i], h0, l0);
+      split_hi_lo(x[2 * i + 1], h1, l1);
+      hb[i] = h0 | (h1 << 16);
+      lb[i] = l0 | (l1 << 16);
     }
-    if (u.param != nullptr) {
-      const float decay = p.decay, ls = u.lr_scale;
-      if (u.param_bf16) {
-        __nv_bfloat16* w = static_cast<__nv_bfloat16*>(u.param) + static_cast<int64_t>(R) * u.ld_param + C0;
-        if (full && u.vec_param) {
-          uint4 raw[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) raw[q] = reinterpret_cast<const uint4*>(w)[q];
-          uint32_t wb[32];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float wf[8];
-            unpack8(raw[q], wf);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) wb[8 * q + e] = float_to_bf16_bits(fmaf(-ls, x[8 * q + e], wf[e] * decay));
-          }
-#pragma unroll
-          for (int q = 0; q < 4; ++q) reinterpret_cast<uint4*>(w)[q] = pack8(wb + 8 * q);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (C0 + j < cols) put_bf16(w + j, float_to_bf16_bits(fmaf(-ls, x[j], bf16_at(w + j) * decay)));
-        }
-      } else {
-        float* w = static_cast<float*>(u.param) + static_cast<int64_t>(R) * u.ld_param + C0;
-        if (full && u.vec_param) {
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            float4 t = reinterpret_cast<float4*>(w)[q];
-            t.x = fmaf(-ls, x[4 * q], t.x * decay);
-            t.y = fmaf(-ls, x[4 * q + 1], t.y * decay);
-            t.z = fmaf(-ls, x[4 * q + 2], t.z * decay);
-            t.w = fmaf(-ls, x[4 * q + 3], t.w * decay);
-            reinterpret_cast<float4*>(w)[q] = t;
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (C0 + j < cols) w[j] = fmaf(-ls, x[j], w[j] * decay);
-        }
-      }
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t o = region_chunk(r, (c0 >> 3) + q);
+      *reinterpret_cast<uint4*>(hib + o) = make_uint4(hb[4 * q], hb[4 * q + 1], hb[4 * q + 2], hb[4 * q + 3]);
+      *reinterpret_cast<uint4*>(lob + o) = make_uint4(lb[4 * q], lb[4 * q + 1], lb[4 * q + 2], lb[4 * q + 3]);
     }
+  } else {
+    write_update<MODE>(p, cd, tl, rank, r, c0, x);
   }
 }
 
 // ------------------------------------------------------------------ the kernel
 
-template <int MODE>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE>::kThreads, 1)
+template <int MODE, bool SMALL>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kThreads, 1)
     muon_ns_gemm_kernel(const __grid_constant__ typename ParamsOf<MODE>::type p) {
-  using L = Lay<MODE>;
+  using L = Lay<MODE, SMALL>;
   constexpr int S = L::S;
   constexpr bool kSym = L::kSym;
   constexpr int NT = L::kEpiThreads;
@@ -367,11 +464,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE>::kThreads,
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + 2;  // used in the leader CTA: both CTAs' epilogues arrive
   uint64_t* tdown = tempty + 2;
-  uint64_t* efull = tdown + 1;  // this CTA's epilogue inputs landed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(efull + 1);
+  uint64_t* efull = tdown + 1;  // staged variant: the tile's hi/lo inputs have landed
+  uint64_t* pdone = efull + 1;  // used in the leader CTA: the peer's producer has finished
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pdone + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* epi_flag = abort_flag + 1;
+  volatile uint32_t* peer_issued = reinterpret_cast<volatile uint32_t*>(epi_flag + 1);  // leader CTA
 
+  griddep_launch_dependents();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int rank = static_cast<int>(cluster_rank());
@@ -390,6 +490,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE>::kThreads,
     }
     mbar_init(tdown, 1);
     mbar_init(efull, 1);
+    mbar_init(pdone, 1);
     *abort_flag = 0;
     *epi_flag = 0;
     fence_mbar_init();
@@ -398,6 +499,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE>::kThreads,
     for (int c = 0; c < p.num_classes; ++c) {
       tma_prefetch_desc(&p.map_a[c]);
       tma_prefetch_desc(&p.map_b[c]);
+      if (SMALL) {
+        tma_prefetch_desc(&p.map_in[c]);
+        tma_prefetch_desc(&p.map_out2[c]);
+      }
     }
   }
   if (warp == 1) {
@@ -411,22 +516,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE>::kThreads,
   const uint32_t tmem_base = *tmem_slot;
   const Watchdog wd{abort_flag, p.status, p.timeout_ns};
   const unsigned long long tb = teardown_budget(p.timeout_ns);
+  griddep_wait();  // operands and scales come from the previous kernel of the step
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer (both CTAs)
+    // Stage-loads are numbered in issue order; load i uses stage i % S in phase i / S.  The
+    // leader arms each phase for both CTAs' bytes.  After a timeout the two producers may
+    // stop at different counts, so the peer reports its count and the leader settles every
+    // phase still open before the CTAs part (see settle below).
     if (lane == 0) {
       const uint32_t full0 = map_to_rank(smem_u32(full), 0);
       int s = 0;
       uint32_t ph = 0;
-      uint32_t armed = 0, armed_par = 0;
+      uint32_t issued = 0;
       bool ok = true;
       for (int t = pair; ok && t < p.total_tiles; t += npairs) {
         const Tile tl = decode_tile<MODE>(p, t);
         const ClassDesc& cd = p.cls[tl.cls];
-        const int row0 = L::TM * tl.I + kBM * rank;
         const CUtensorMap* ma = &p.map_a[tl.cls];
         const CUtensorMap* mb = &p.map_b[tl.cls];
-        const int nk = (cd.ksize + kBK - 1) / kBK;
+        const int nk = (cd.ksize + L::BK - 1) / L::BK;
+        const int a0 = L::TM * tl.I + kBM * rank;
         const int b0 = L::TN * tl.J + kBM * rank;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1u, wd, kSiteProducerEmpty)) {
@@ -437,26 +547,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE>::kThreads,
           uint8_t* sb = sa + L::kABytes;
           if (leader_cta) mbar_arrive_expect_tx(&full[s], 2 * L::kStageBytes);
           const uint32_t fb = full0 + 8u * static_cast<uint32_t>(s);
-          const int k0 = kb * kBK;
-#pragma unroll
-          for (int b = 0; b < kBM / kBox; ++b) load_box_pair(sa + b * kBoxBytes, ma, cd.a_mn, row0 + b * kBox, k0, tl.mat, fb);
-#pragma unroll
-          for (int b = 0; b < kBM / kBox; ++b) load_box_pair(sb + b * kBoxBytes, mb, cd.b_mn, b0 + b * kBox, k0, tl.mat, fb);
-          armed |= 1u << s;
-          armed_par = (armed_par & ~(1u << s)) | (ph << s);
+          const int k0 = kb * L::BK;
+          constexpr int kPart = L::kABytes / 2;
+          load_half_pair<L::BK>(sa, ma, cd.a_mn, a0, k0, 0, tl.mat, fb);
+          load_half_pair<L::BK>(sa + kPart, ma, cd.a_mn, a0, k0, 1, tl.mat, fb);
+          load_half_pair<L::BK>(sb, mb, cd.b_mn, b0, k0, 0, tl.mat, fb);
+          load_half_pair<L::BK>(sb + kPart, mb, cd.b_mn, b0, k0, 1, tl.mat, fb);
+          ++issued;
           if (++s == S) {
             s = 0;
             ph ^= 1u;
           }
         }
       }
-      if (!ok) {
-        // Do not leave while a load may still write into shared memory.  The peer's
-        // operand bytes complete on the leader's barriers, which the leader waits for
-        // here; the final cluster barrier keeps the peer until then.
-        if (leader_cta)
-          for (int j = 0; j < S; ++j)
-            if (armed & (1u << j)) quiet_wait(&full[j], (armed_par >> j) & 1u, tb);
+      if (!leader_cta) {
+        st_cluster_u32(map_to_rank(smem_u32(const_cast<uint32_t*>(peer_issued)), 0), issued);
+        mbar_arrive_cluster(map_to_rank(smem_u32(pdone), 0));
+      } else {
+        // Settle.  A load i below min(nL, nP) - S has completed: both producers waited for
+        // stage i % S to be consumed again.  Each remaining i, in order, is waited for after
+        //   i < nL, i < nP : nothing (armed, both shares issued)
+        //   i < nL, i >= nP: completing the peer's share, which will never be sent
+        //   i >= nL, i < nP: arming the phase for the peer's share alone
+        // so no copy is in flight into either CTA when the final cluster barrier opens.
+        // Phase i of a stage completes before load i + S of it is issued, so every wait
+        // below is for the stage's current phase.
+        const uint32_t nl = issued;
+        uint32_t np = nl;
+        bool known = false;
+        {
+          const uint64_t t0 = global_timer_ns();
+          while (!(known = mbar_try_wait_cluster(pdone, 0)) && global_timer_ns() - t0 < tb) {
+          }
+          if (known) np = *peer_issued;
+        }
+        const uint32_t both = nl < np ? nl : np;
+        const uint32_t lo_i = both >= static_cast<uint32_t>(S) ? both - S : 0u;
+        const uint32_t hi_i = nl > np ? nl : np;
+        for (uint32_t i = lo_i; i < hi_i; ++i) {
+          const int st = static_cast<int>(i % S);
+          const uint32_t par = (i / S) & 1u;
+          if (i >= nl)
+            mbar_arrive_expect_tx(&full[st], L::kStageBytes);
+          else if (i >= np)
+            mbar_complete_tx(&full[st], L::kStageBytes);
+          quiet_wait(&full[st], par, tb);
+        }
       }
     }
   } else if (warp == 1) {
@@ -469,7 +605,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE>::kThreads,
         for (int t = pair; ok && t < p.total_tiles; t += npairs) {
           const Tile tl = decode_tile<MODE>(p, t);
           const ClassDesc& cd = p.cls[tl.cls];
-          const int nk = (cd.ksize + kBK - 1) / kBK;
+          const int nk = (cd.ksize + L::BK - 1) / L::BK;
           const uint32_t idesc = idesc_bf16_f32(L::TM, L::TN, cd.a_mn, cd.b_mn);
           if (!mbar_wait(&tempty[acc], aph ^ 1u, wd, kSiteMmaTmemEmpty)) break;
           tc_fence_after();
@@ -483,8 +619,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE>::kThreads,
             const uint32_t sa = smem_u32(smem + s * L::kStageBytes);
             const uint32_t sb = sa + L::kABytes;
 #pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk)
-              umma_bf16_pair(dtm, operand_desc(sa, cd.a_mn, kk), operand_desc(sb, cd.b_mn, kk), idesc,
+            for (int kk = 0; kk < L::BK / 16; ++kk)
+              umma_bf16_pair(dtm, operand_desc<L::BK>(sa, cd.a_mn, kk), operand_desc<L::BK>(sb, cd.b_mn, kk), idesc,
                              (kb | kk) != 0 ? 1u : 0u);
             umma_commit_pair(&empty[s], 0x3);
             if (++s == S) {
@@ -505,127 +641,79 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE>::kThreads,
       }
       quiet_wait(tdown, 0, tb);
     }
-  } else {
-    // ---------------------------------------------------------------- epilogue (both CTAs)
+  } else if constexpr (SMALL) {
+    // ---------------------------------------------------------------- staged apply epilogue (both CTAs)
+    // The tile's old hi/lo (128 x 256 each per CTA) are loaded by TMA into the staging
+    // region by the epilogue leader as soon as the previous tile is done with it, so they
+    // are in place before the accumulator is; kApply updates them in place and stores
+    // them back by TMA, one 128-column half at a time.
     const int ew = warp - 2;
-    const int q = warp & 3;  // TMEM lanes 32q..32q+31 belong to this warp
-    const int h = ew >> 2;   // column group within a 128-column block
-    const int r = q * 32 + lane;
+    const int q4 = warp & 3;  // TMEM lanes 32 q4 .. 32 q4 + 31 belong to this warp
+    const int h = ew >> 2;    // which 64 columns of each 128-column half
+    const int r = q4 * 32 + lane;
     const bool leader = threadIdx.x == 64;
     const uint32_t tempty0 = map_to_rank(smem_u32(tempty), 0);
-    uint8_t* D = epi;
-    uint8_t* T = epi + L::kBlk;
-    uint8_t* Ain = epi + 2 * L::kBlk;
+    uint8_t* hib = epi;
+    uint8_t* lob = epi + 4 * L::kHalf;
     int acc = 0;
     uint32_t aph = 0;
-    // Epilogue inputs (polynomial: A; apply: hi and lo) for tile t are loaded by the
-    // epilogue leader as soon as tile t - 1 no longer needs the buffer, so the main
-    // loop never waits on them.
-    bool in_pending = false;
+    bool in_pending = false;  // leader: a load into the region has not been waited for
     uint32_t in_par = 0;
-    auto load_inputs = [&](int tt) {
+    auto load_inputs = [&](int tt, uint32_t par) {
       const Tile nx = decode_tile<MODE>(p, tt);
       const int row0 = L::TM * nx.I + kBM * rank, col0 = L::TN * nx.J;
-      fence_proxy_async_smem();
-      if constexpr (MODE == kPoly) {
-        mbar_arrive_expect_tx(efull, 2 * L::kBlk);
-        load_region<4>(Ain, &p.map_in0[nx.cls], efull, row0, col0, nx.mat);
-      } else {
-        mbar_arrive_expect_tx(efull, 4 * L::kBlk);
-        load_region<4>(epi, &p.map_in0[nx.cls], efull, row0, col0, nx.mat);
-        load_region<4>(epi + 2 * L::kBlk, &p.map_in1[nx.cls], efull, row0, col0, nx.mat);
-      }
+      mbar_arrive_expect_tx(efull, 8 * L::kHalf);
+      load_region(hib, &p.map_in[nx.cls], efull, row0, col0, nx.mat);
+      load_region(lob, &p.map_out2[nx.cls], efull, row0, col0, nx.mat);
       in_pending = true;
+      in_par = par;
     };
-    if (MODE != kGram && leader && pair < p.total_tiles) load_inputs(pair);
+    if (leader && pair < p.total_tiles) load_inputs(pair, 0u);
     int k = 0;
     for (int t = pair; t < p.total_tiles; t += npairs, ++k) {
       const Tile tl = decode_tile<MODE>(p, t);
       const ClassDesc& cd = p.cls[tl.cls];
       const uint32_t kpar = static_cast<uint32_t>(k) & 1u;
-      // One warp waits for the accumulator (and the staged inputs); the rest learn the
-      // outcome at the barrier, so every epilogue warp leaves the loop together.
       if (ew == 0) {
         bool ok = warp_wait(&tfull[acc], aph, wd, kSiteEpilogueFull);
-        if (ok && MODE != kGram) ok = warp_wait(efull, kpar, wd, kSiteEpilogueIn);
+        if (ok) ok = warp_wait(efull, kpar, wd, kSiteEpilogueIn);
         if (lane == 0) *epi_flag = ok ? 1 : 0;
       }
       named_barrier(1, NT);
       if (*epi_flag == 0) break;
-      if (MODE != kGram) {
-        in_pending = false;
-        in_par = kpar ^ 1u;
-      }
+      in_pending = false;
       tc_fence_after();
-      const uint32_t tacc = tmem_base + static_cast<uint32_t>(acc * L::TN) + (static_cast<uint32_t>(q * 32) << 16);
-      if constexpr (kSym) {
-        const int rb = 2 * tl.I + rank;  // this CTA's 128-row block
-        float mul = 1.f;
-        if (MODE == kGram && p.first_iter) {
-          const float sv = p.scale[cd.mat_base + tl.mat];
-          mul = sv * sv;
-        }
-        bool stored = false;
+      const uint32_t tacc = tmem_base + static_cast<uint32_t>(acc * L::TN) + (static_cast<uint32_t>(q4 * 32) << 16);
+      const float sc = p.first_iter ? p.scale[cd.mat_base + tl.mat] : 1.f;
+      const int row0 = L::TM * tl.I + kBM * rank, col0 = L::TN * tl.J;
 #pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {
-          const int cb = 2 * tl.J + hh;
-          if (rb > cb) continue;  // below the diagonal: its mirror is stored by another block
-          if (stored) {
-            if (leader) bulk_wait_read<0>();
-            named_barrier(1, NT);  // D and T free again
-          }
-          sym_block<MODE>(p, mul, rb == cb, r, h, hh, tacc, D, T, Ain);
+      for (int hh = 0; hh < 2; ++hh) {
+        const int c0 = 128 * hh + 64 * h;
+        apply_staged<MODE>(p, cd, tl, rank, r, c0, tacc + c0, hib, lob, sc);
+        apply_staged<MODE>(p, cd, tl, rank, r, c0 + 32, tacc + c0 + 32, hib, lob, sc);
+        if (hh == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * static_cast<uint32_t>(acc));
+        }
+        if constexpr (MODE == kApply) {
           fence_proxy_async_smem();
           named_barrier(1, NT);
           if (leader) {
-            const CUtensorMap* mo = &p.map_out[tl.cls];
-            store_region<2>(mo, D, 0, 2, kBM * rb, kBM * cb, tl.mat);
-            if (rb < cb) store_region<2>(mo, T, 0, 2, kBM * cb, kBM * rb, tl.mat);
+            store_region(&p.map_out[tl.cls], hib, 2 * hh, 2, row0, col0, tl.mat);
+            store_region(&p.map_out2[tl.cls], lob, 2 * hh, 2, row0, col0, tl.mat);
             bulk_commit();
           }
-          stored = true;
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * static_cast<uint32_t>(acc));
-        if (leader) {
-          if (MODE == kPoly && t + npairs < p.total_tiles) load_inputs(t + npairs);
-          bulk_wait_read<0>();  // D and T are free for the next tile
-        }
-      } else {
-        uint8_t* hib = epi;
-        uint8_t* lob = epi + 2 * L::kBlk;
-        const float sc = p.first_iter ? p.scale[cd.mat_base + tl.mat] : 1.f;
-#pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {
-          apply_cols<MODE>(p, cd, tl, rank, r, 128 * hh + 64 * h, tacc, hib, lob, sc);
-          apply_cols<MODE>(p, cd, tl, rank, r, 128 * hh + 64 * h + 32, tacc, hib, lob, sc);
-          if (hh == 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * static_cast<uint32_t>(acc));
-          }
-          if constexpr (MODE == kApply) {
-            fence_proxy_async_smem();
-            named_barrier(1, NT);
-            if (leader) {
-              const int row0 = L::TM * tl.I + kBM * rank, col0 = L::TN * tl.J;
-              store_region<4>(&p.map_out[tl.cls], hib, 2 * hh, 2, row0, col0, tl.mat);
-              store_region<4>(&p.map_in1[tl.cls], lob, 2 * hh, 2, row0, col0, tl.mat);
-              bulk_commit();
-            }
-          }
-        }
-        if constexpr (MODE == kApply) {
-          if (leader) {
-            bulk_wait_read<0>();  // the stores have read the region: it can be refilled
-            if (t + npairs < p.total_tiles) load_inputs(t + npairs);
-          }
-        } else {
-          named_barrier(1, NT);  // every thread is done reading the input region
-          if (leader && t + npairs < p.total_tiles) load_inputs(t + npairs);
         }
       }
+      // the region is refilled once nothing reads it any more
+      if constexpr (MODE == kApply) {
+        if (leader) bulk_wait_read<0>();
+      } else {
+        fence_proxy_async_smem();
+        named_barrier(1, NT);
+      }
+      if (leader && t + npairs < p.total_tiles) load_inputs(t + npairs, kpar ^ 1u);
       if (++acc == 2) {
         acc = 0;
         aph ^= 1u;
@@ -635,6 +723,148 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE>::kThreads,
       bulk_wait_all();
       if (in_pending) quiet_wait(efull, in_par, tb);
     }
+  } else {
+    // ---------------------------------------------------------------- epilogue (both CTAs)
+    const int ew = warp - 2;
+    const int q4 = warp & 3;  // TMEM lanes 32 q4 .. 32 q4 + 31 belong to this warp
+    const int h = ew >> 2;    // which 32 columns of each 64-column quarter
+    const int r = q4 * 32 + lane;
+    const bool leader = threadIdx.x == 64;
+    const uint32_t tempty0 = map_to_rank(smem_u32(tempty), 0);
+    uint8_t* Q = epi;
+    uint8_t* Tst = epi + L::kHalf;
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int t = pair; t < p.total_tiles; t += npairs) {
+      const Tile tl = decode_tile<MODE>(p, t);
+      const ClassDesc& cd = p.cls[tl.cls];
+      // Epilogue inputs come straight from global memory (L2) into registers; they are
+      // requested before the accumulator is waited for.
+      uint4 in_a[4][4];  // polynomial: A, the four quarters' 32 columns of this row
+      uint4 ch[4], cl[4];  // apply: hi and lo of the first quarter
+      const int rb = 2 * tl.I + rank;
+      const int Rx = L::TM * tl.I + kBM * rank + r;
+      const int64_t xoff = tl.mat * cd.x_stride + static_cast<int64_t>(Rx) * cd.ldx;
+      const int Cb = L::TN * tl.J + 32 * h;
+      if constexpr (MODE == kPoly) {
+        const int Ra = kBM * rb + r;
+        const __nv_bfloat16* arow = cd.a_buf + tl.mat * cd.a_stride + static_cast<int64_t>(Ra) * cd.lda;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int cb = 2 * tl.J + (q >> 1);
+          const int C = Cb + 64 * q;
+          load_row32(arow + C, cd.m - C, Ra < cd.m && rb <= cb, in_a[q]);
+        }
+      } else if constexpr (!kSym) {
+        load_row32(cd.x_hi_cur + xoff + Cb, cd.cols - Cb, Rx < cd.rows, ch);
+        load_row32(cd.x_lo + xoff + Cb, cd.cols - Cb, Rx < cd.rows, cl);
+      }
+      // The next tile's epilogue inputs start moving from HBM into L2 now, so that its
+      // loads above hit L2 (apply: hi and lo; polynomial: A).
+      if (MODE != kGram && leader && t + npairs < p.total_tiles) {
+        const Tile nx = decode_tile<MODE>(p, t + npairs);
+        const ClassDesc& nd = p.cls[nx.cls];
+        if constexpr (MODE == kPoly) {
+          const int rbn = 2 * nx.I + rank;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tma_prefetch_l2_3d(&p.map_a[nx.cls], L::TN * nx.J + 64 * c, kBM * rbn, nx.mat);
+        } else {
+          const int rn = L::TM * nx.I + kBM * rank;
+          const CUtensorMap* mh = nd.tall ? &p.map_a[nx.cls] : &p.map_b[nx.cls];  // the operand map of hi
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            tma_prefetch_l2_3d(mh, L::TN * nx.J + 64 * c, rn, nx.mat);
+            tma_prefetch_l2_3d(&p.map_out2[nx.cls], L::TN * nx.J + 64 * c, rn, nx.mat);
+            tma_prefetch_l2_3d(&p.map_out2[nx.cls], L::TN * nx.J + 64 * c, rn + 64, nx.mat);
+          }
+        }
+      }
+      // One warp waits for the accumulator; the rest learn the outcome at the barrier, so
+      // every epilogue warp leaves the loop together.
+      if (ew == 0) {
+        const bool ok = warp_wait(&tfull[acc], aph, wd, kSiteEpilogueFull);
+        if (lane == 0) *epi_flag = ok ? 1 : 0;
+      }
+      named_barrier(1, NT);
+      if (*epi_flag == 0) break;
+      tc_fence_after();
+      const uint32_t tacc = tmem_base + static_cast<uint32_t>(acc * L::TN) + (static_cast<uint32_t>(q4 * 32) << 16);
+      if constexpr (kSym) {
+        float mul = 1.f;
+        if (MODE == kGram && p.first_iter) {
+          const float sv = p.scale[cd.mat_base + tl.mat];
+          mul = sv * sv;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int cb = 2 * tl.J + (q >> 1);
+          if (rb > cb) continue;  // below the diagonal: stored by the block's mirror
+          if (leader) bulk_wait_read<0>();
+          named_barrier(1, NT);  // staging free
+          sym_quarter<MODE>(p, mul, rb == cb, r, h, tacc + 64 * q + 32 * h, Q, Tst, in_a[q]);
+          if (q == 3) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * static_cast<uint32_t>(acc));
+          }
+          fence_proxy_async_smem();
+          named_barrier(1, NT);
+          if (leader) {
+            store_q(&p.map_out[tl.cls], Q, kBM * rb, kBM * cb + 64 * (q & 1), tl.mat);
+            if (rb != cb) store_t(&p.map_out[tl.cls], Tst, kBM * cb + 64 * (q & 1), kBM * rb, tl.mat);
+            bulk_commit();
+          }
+        }
+      } else {
+        const float sc = p.first_iter ? p.scale[cd.mat_base + tl.mat] : 1.f;
+        const int row0 = L::TM * tl.I + kBM * rank;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 nh[4], nl[4];
+          if (q < 3) {
+            const int Cn = Cb + 64 * (q + 1);
+            load_row32(cd.x_hi_cur + xoff + Cn, cd.cols - Cn, Rx < cd.rows, nh);
+            load_row32(cd.x_lo + xoff + Cn, cd.cols - Cn, Rx < cd.rows, nl);
+          }
+          uint32_t hb[16], lb[16];
+          apply_quarter<MODE>(p, cd, tl, rank, r, 64 * q + 32 * h, tacc + 64 * q + 32 * h, ch, cl, sc, hb, lb);
+          if (q == 3) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * static_cast<uint32_t>(acc));
+          }
+          if constexpr (MODE == kApply) {
+            if (leader) bulk_wait_read<0>();
+            named_barrier(1, NT);  // staging free
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint32_t o = q_chunk(r, 4 * h + k);
+              *reinterpret_cast<uint4*>(Q + o) = make_uint4(hb[4 * k], hb[4 * k + 1], hb[4 * k + 2], hb[4 * k + 3]);
+              *reinterpret_cast<uint4*>(Tst + o) = make_uint4(lb[4 * k], lb[4 * k + 1], lb[4 * k + 2], lb[4 * k + 3]);
+            }
+            fence_proxy_async_smem();
+            named_barrier(1, NT);
+            if (leader) {
+              store_q(&p.map_out[tl.cls], Q, row0, L::TN * tl.J + 64 * q, tl.mat);
+              store_q(&p.map_out2[tl.cls], Tst, row0, L::TN * tl.J + 64 * q, tl.mat);
+              bulk_commit();
+            }
+          }
+          if (q < 3) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              ch[k] = nh[k];
+              cl[k] = nl[k];
+            }
+          }
+        }
+      }
+      if (++acc == 2) {
+        acc = 0;
+        aph ^= 1u;
+      }
+    }
+    if (leader) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -646,42 +876,59 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE>::kThreads,
   }
 }
 
-template <int MODE>
+template <int MODE, bool SMALL>
 static cudaError_t launch_one(const typename ParamsOf<MODE>::type& p, int max_pairs, cudaStream_t stream) {
-  using L = Lay<MODE>;
+  using L = Lay<MODE, SMALL>;
+  auto* kernel = muon_ns_gemm_kernel<MODE, SMALL>;
   static thread_local int configured_device = -1;
   static thread_local int resident_pairs = 0;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (configured_device != dev) {
-    e = cudaFuncSetAttribute(muon_ns_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * max_pairs, 1, 1);
     cfg.blockDim = dim3(L::kThreads, 1, 1);
     cfg.dynamicSmemBytes = L::kSmemBytes;
     int clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&clusters, muon_ns_gemm_kernel<MODE>, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg);
     if (e != cudaSuccess) return e;
     resident_pairs = clusters > 0 ? clusters : 1;
     configured_device = dev;
   }
   const int pairs = std::max(1, std::min(std::min(p.total_tiles, max_pairs), resident_pairs));
-  muon_ns_gemm_kernel<MODE><<<2 * pairs, L::kThreads, L::kSmemBytes, stream>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(L::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = L::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
 int gemm_tile_rows() { return 256; }
 int gemm_tile_cols() { return 256; }
 
-// `max_pairs` bounds the number of CTA pairs (half the SM count).
+// `max_pairs` bounds the number of CTA pairs (half the SM count).  Apply launches with
+// p->staged set run the staged variant, whose operand maps have 64 x 64 boxes.
 cudaError_t launch_gemm(int mode, const GemmParams* p, int max_pairs, cudaStream_t stream) {
   switch (mode) {
-    case kGram: return launch_one<kGram>(*p, max_pairs, stream);
-    case kPoly: return launch_one<kPoly>(*p, max_pairs, stream);
-    case kApply: return launch_one<kApply>(*p, max_pairs, stream);
-    case kApplyLast: return launch_one<kApplyLast>(*static_cast<const FinalParams*>(p), max_pairs, stream);
+    case kGram: return launch_one<kGram, false>(*p, max_pairs, stream);
+    case kPoly: return launch_one<kPoly, false>(*p, max_pairs, stream);
+    case kApply:
+      return p->staged ? launch_one<kApply, true>(*p, max_pairs, stream)
+                       : launch_one<kApply, false>(*p, max_pairs, stream);
+    case kApplyLast: {
+      const FinalParams& f = *static_cast<const FinalParams*>(p);
+      return p->staged ? launch_one<kApplyLast, true>(f, max_pairs, stream)
+                       : launch_one<kApplyLast, false>(f, max_pairs, stream);
+    }
     default: return cudaErrorInvalidValue;
   }
 }

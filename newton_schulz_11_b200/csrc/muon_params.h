@@ -14,9 +14,7 @@ namespace muon {
 constexpr int kMaxClasses = 8;      // distinct shapes per wave
 constexpr int kMaxWaveMats = 128;   // matrices per wave
 constexpr int kBM = 128;            // tile rows = UMMA M
-constexpr int kBK = 64;             // k-block: one 128-byte swizzled row of bf16
-constexpr int kBox = 64;            // TMA box edge (elements); every box is 64 x 64 bf16
-constexpr int kBoxBytes = kBox * kBox * 2;
+constexpr int kBox = 64;            // TMA box inner edge (elements, 128 bytes of bf16)
 
 enum GemmMode : int {
   kGram = 0,       // A = s^2 X X^T (iteration 0) or X X^T, upper tiles, mirrored store
@@ -74,14 +72,15 @@ struct UpdMat {
 };
 
 struct GemmParams {
-  CUtensorMap map_a[kMaxClasses];   // operand A of the launch, per class
-  CUtensorMap map_b[kMaxClasses];   // operand B
-  CUtensorMap map_in0[kMaxClasses];  // epilogue input: apply -> hi of X, polynomial -> A
-  CUtensorMap map_in1[kMaxClasses];  // epilogue input: apply -> lo of X (written back in place)
-  CUtensorMap map_out[kMaxClasses];  // epilogue output: Gram -> A, polynomial -> B, apply -> next hi
+  CUtensorMap map_a[kMaxClasses];     // operand A of the launch, per class (64 x 128 boxes)
+  CUtensorMap map_b[kMaxClasses];     // operand B (64 x 128 boxes)
+  CUtensorMap map_out[kMaxClasses];   // epilogue store: Gram -> A, polynomial -> B, apply -> next hi
+  CUtensorMap map_out2[kMaxClasses];  // epilogue store: apply -> lo (64 x 64 boxes, like map_out)
+  CUtensorMap map_in[kMaxClasses];    // staged apply: the current hi as epilogue input (64 x 64)
   ClassDesc cls[kMaxClasses];
   int32_t num_classes;
   int32_t total_tiles;
+  int32_t staged;                   // apply: the staged variant (operand maps with 64 x 64 boxes)
   int32_t first_iter;               // iteration 0: s^2 on the Gram, s on the apply
   float a, b, c;                    // this iteration's coefficients
   float decay;                      // 1 - lr * weight_decay (final epilogue)
