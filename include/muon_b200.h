@@ -69,7 +69,9 @@ typedef enum {
   MUON_ERR_WORKSPACE_TOO_SMALL = 5,/* not even the largest single matrix fits */
   MUON_ERR_CUDA = 6,               /* a CUDA runtime call or launch failed */
   MUON_ERR_TIMEOUT = 7,            /* device status only: a bounded wait ran out */
-  MUON_ERR_NO_DEVICE = 8           /* current device is not an sm_100 GPU */
+  MUON_ERR_NO_DEVICE = 8,          /* current device is not an sm_100 GPU */
+  MUON_ERR_STATIC_SCRATCH_LIMIT = 9 /* muon_newton_schulz_static: a matrix needs more
+                                       scratch than MUON_STATIC_SCRATCH_BYTES */
 } muon_status_t;
 
 typedef enum { MUON_F32 = 0, MUON_BF16 = 1 } muon_dtype_t;
@@ -182,6 +184,39 @@ muon_status_t muon_set_wait_timeout_us(int64_t us);
 
 muon_status_t muon_profile_begin(void);
 muon_status_t muon_profile_end(double* ms_by_kind, int64_t* launches_by_kind, int kinds);
+
+/*
+ * Newton-Schulz without a caller-supplied workspace, for callers that cannot allocate
+ * device memory: code that runs inside another framework's memory pool or allocator
+ * (where a cudaMalloc of its own would fragment that pool, or is forbidden), plugins
+ * and embedded hosts that only receive ready-made device buffers, and callers that
+ * must not allocate between steps.  There is no counterpart in the paper; this is a
+ * packaging of muon_newton_schulz.
+ *
+ * Same arguments and results as muon_newton_schulz, except that the scratch is a
+ * static device array of MUON_STATIC_SCRATCH_BYTES inside this library.  Every GPU
+ * that loads the library holds that array until the process exits.  The call
+ * allocates no device memory: no cudaMalloc or cudaFree, no allocating library.
+ *
+ *   - A matrix whose own scratch (hi/lo copies, Gram and polynomial buffers) does not
+ *     fit in MUON_STATIC_SCRATCH_BYTES is rejected with MUON_ERR_STATIC_SCRATCH_LIMIT
+ *     before anything is queued.  Sets that fit only together are processed in waves.
+ *   - The first call on a device looks up the array's device address with the
+ *     device current (cudaGetSymbolAddress).  Make that first call outside any
+ *     stream capture.
+ *   - All calls share the one array, which keeps the last call's contents.  Each call
+ *     clears the array's status word before its kernels run.  Calls whose kernels
+ *     overlap on the GPU (other streams, other host threads) race on the array and
+ *     give wrong results: keep them ordered, e.g. on one stream.
+ *   - device_status (may be NULL): 2 int32 in device or pinned host memory; after the
+ *     call's kernels, in stream order, it receives the status word (MUON_OK or
+ *     MUON_ERR_TIMEOUT) and the wait that gave up, as muon_device_status reports them.
+ */
+#define MUON_STATIC_SCRATCH_BYTES (64u << 20)
+
+muon_status_t muon_newton_schulz_static(const muon_matrix_t* mats, int n, int ns_steps,
+                                        const float* coeffs, float eps, int32_t* device_status,
+                                        void* stream);
 
 #ifdef __cplusplus
 }

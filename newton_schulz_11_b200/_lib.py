@@ -17,6 +17,8 @@ MUON_ERR_WORKSPACE_TOO_SMALL = 5
 MUON_ERR_CUDA = 6
 MUON_ERR_TIMEOUT = 7
 MUON_ERR_NO_DEVICE = 8
+MUON_ERR_STATIC_SCRATCH_LIMIT = 9
+MUON_STATIC_SCRATCH_BYTES = 64 << 20
 
 MUON_F32 = 0
 MUON_BF16 = 1
@@ -34,6 +36,7 @@ EXPORTS = (
     "muon_set_wait_timeout_us",
     "muon_profile_begin",
     "muon_profile_end",
+    "muon_newton_schulz_static",
 )
 
 KIND_NAMES = ("momentum", "norm", "gram", "poly", "apply", "apply_last")
@@ -127,6 +130,9 @@ def lib() -> ctypes.CDLL:
         h.muon_profile_begin.argtypes = []
         h.muon_profile_end.restype = ctypes.c_int
         h.muon_profile_end.argtypes = [P(ctypes.c_double), P(ctypes.c_int64), ctypes.c_int]
+        h.muon_newton_schulz_static.restype = ctypes.c_int
+        h.muon_newton_schulz_static.argtypes = [P(MuonMatrix), ctypes.c_int, ctypes.c_int, P(ctypes.c_float),
+                                                ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p]
         _lib = h
         return h
 

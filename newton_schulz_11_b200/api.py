@@ -183,6 +183,33 @@ def newton_schulz(Gs: Sequence[torch.Tensor], *, coeffs=None, eps: float = DEFAU
     return outs
 
 
+def newton_schulz_static(Gs: Sequence[torch.Tensor], *, coeffs=None, eps: float = DEFAULT_EPS, outs=None,
+                         device_status: Optional[torch.Tensor] = None, stream=None) -> List[torch.Tensor]:
+    """newton_schulz with the library's static device scratch in place of a workspace.
+
+    For callers that cannot allocate device memory of their own.  `outs` (if given) and
+    `device_status` (an int32 tensor of 2, device or pinned host) are the only buffers
+    written; nothing is allocated on the device when `outs` is given.
+    """
+    Gs = list(Gs)
+    if not Gs:
+        raise ValueError("Gs must be a non-empty list")
+    if outs is None:
+        outs = [torch.empty_like(g) for g in Gs]
+    table, steps = _coeff_array(coeffs if coeffs is not None else quintic_table())
+    device = Gs[0].device
+    arr = _descriptors(None, Gs, None, outs, None, ns_only=True)
+    st_ptr = None
+    if device_status is not None:
+        if device_status.dtype != torch.int32 or device_status.numel() < 2 or not device_status.is_contiguous():
+            raise ValueError("device_status must be a contiguous int32 tensor of at least 2 elements")
+        st_ptr = device_status.data_ptr()
+    s = _stream_handle(device, stream)
+    check(lib().muon_newton_schulz_static(arr, len(Gs), steps, table, float(eps), st_ptr, s),
+          "muon_newton_schulz_static")
+    return outs
+
+
 def scratch_view(shapes: Sequence[Tuple[int, int]], index: int, workspace_bytes: int) -> MuonScratchView:
     n = len(shapes)
     arr = (MuonMatrix * n)()

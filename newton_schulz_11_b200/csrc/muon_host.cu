@@ -669,6 +669,7 @@ const char* muon_status_str(int status) {
     case MUON_ERR_CUDA: return "CUDA runtime error";
     case MUON_ERR_TIMEOUT: return "device-side wait timed out";
     case MUON_ERR_NO_DEVICE: return "no sm_100 device is current";
+    case MUON_ERR_STATIC_SCRATCH_LIMIT: return "a matrix needs more scratch than the static array holds (64 MiB)";
     default: return "unknown status";
   }
 }
@@ -789,3 +790,61 @@ muon_status_t muon_profile_end(double* ms_by_kind, int64_t* launches_by_kind, in
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- static scratch
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = MUON_STATIC_SCRATCH_BYTES;
+constexpr int kMaxDevices = 64;
+
+// Scratch of muon_newton_schulz_static.  In host code `g_static_scratch` only names the
+// symbol; its device address comes from cudaGetSymbolAddress, per device.
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+std::mutex g_static_mu;
+void* g_static_addr[kMaxDevices] = {};
+
+// Device address of the array on device `dev`, which is current.  Looked up once.
+muon_status_t static_scratch(int dev, void** addr) {
+  if (dev < 0 || dev >= kMaxDevices) return MUON_ERR_NO_DEVICE;
+  std::lock_guard<std::mutex> lk(g_static_mu);
+  if (g_static_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return MUON_ERR_CUDA;
+    g_static_addr[dev] = p;
+  }
+  *addr = g_static_addr[dev];
+  return MUON_OK;
+}
+
+}  // namespace
+
+extern "C" muon_status_t muon_newton_schulz_static(const muon_matrix_t* mats, int n, int ns_steps,
+                                                   const float* coeffs, float eps, int32_t* device_status,
+                                                   void* stream) {
+  muon_status_t st = validate(mats, n, true);
+  if (st != MUON_OK) return st;
+  st = validate_hyper(0.f, 0.f, 0.f, 0, ns_steps, coeffs, eps);
+  if (st != MUON_OK) return st;
+  {
+    std::vector<WavePlan> waves;
+    st = form_waves(mats, n, kStaticScratchBytes, &waves);
+    if (st == MUON_ERR_WORKSPACE_TOO_SMALL) return MUON_ERR_STATIC_SCRATCH_LIMIT;
+    if (st != MUON_OK) return st;
+  }
+  int dev = 0, sms = 0;
+  st = current_device(&dev, &sms);
+  if (st != MUON_OK) return st;
+  void* ws = nullptr;
+  st = static_scratch(dev, &ws);
+  if (st != MUON_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, kHeaderBytes, s) != cudaSuccess) return MUON_ERR_CUDA;
+  st = run(mats, n, 0.f, 0.f, 0.f, 0, ns_steps, coeffs, eps, ws, kStaticScratchBytes, stream, true);
+  if (st != MUON_OK) return st;
+  if (device_status != nullptr &&
+      cudaMemcpyAsync(device_status, ws, 2 * sizeof(int32_t), cudaMemcpyDefault, s) != cudaSuccess)
+    return MUON_ERR_CUDA;
+  return MUON_OK;
+}
