@@ -68,7 +68,8 @@ def matrix_work(rows, cols):
 
 
 def kind_bytes(w, kind, with_out=False):
-    """Algorithmic HBM bytes of one launch of `kind` over the whole workload."""
+    """Algorithmic HBM bytes of one launch of `kind` over the whole workload: every input
+    the launch needs read once, every output written once (X is a bf16 hi/lo pair)."""
     pb = 2 if w.param_dtype == "bf16" else 4
     tot = 0
     for rows, cols in w.shapes:
@@ -79,13 +80,13 @@ def kind_bytes(w, kind, with_out=False):
         elif kind == "norm":
             tot += 0
         elif kind == "gram":
-            tot += 2 * mn + 2 * m * m
+            tot += 2 * mn + 2 * m * m    # read hi; write A
         elif kind == "poly":
-            tot += 6 * m * m         # A operand, A in the epilogue, B out
+            tot += 4 * m * m             # read A; write B
         elif kind == "apply":
-            tot += 10 * mn + 2 * m * m   # hi operand + hi, lo in, hi, lo out; B operand
+            tot += 8 * mn + 2 * m * m    # read hi, lo and B; write hi, lo
         elif kind == "apply_last":
-            tot += (6 + 2 * pb + (4 if with_out else 0)) * mn + 2 * m * m
+            tot += (4 + 2 * pb + (4 if with_out else 0)) * mn + 2 * m * m   # read hi, lo, B; W in/out; O
     return tot
 
 
@@ -232,7 +233,9 @@ def load_coeffs(w):
 
 # ------------------------------------------------------------------ distributed plumbing
 
-def dist_setup(args):
+def dist_setup(args, backend=None):
+    """One process per GPU (torchrun env).  NCCL on GPUs; `backend="gloo"` runs the same
+    rank logic on CPU processes (tests)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -240,19 +243,25 @@ def dist_setup(args):
         import torch
         import torch.distributed as dist
 
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        backend = backend or "nccl"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
     return world, rank, local
 
 
 def dist_max(x, world):
+    """Max of a per-rank number over all ranks (every rank gets it)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -266,18 +275,59 @@ def barrier(world):
 
 # ------------------------------------------------------------------ reference arm
 
+def oracle_step_samples(w):
+    """One bounded sample per reference step: the fp64 oracle's step on ONE matrix,
+    cycling through the workload's distinct shapes; each sample is scaled to a full step
+    by the work ratio (algorithmic NS flops plus elementwise elements) of the whole
+    workload to that matrix.  Yields (ms per full step, shape)."""
+    import numpy as np
+
+    import oracle
+
+    coeffs = load_coeffs(w)
+    by_shape = {}
+    for i, s in enumerate(w.shapes):
+        by_shape.setdefault(s, []).append(i)
+
+    def work(r, c):
+        mw = matrix_work(r, c)
+        return (mw["gram"] + mw["poly"] + mw["apply"]) * w.ns_steps + 16 * r * c
+
+    total = sum(work(r, c) for r, c in w.shapes)
+    shapes = list(by_shape)
+    step = inputs.first_step_index(w)
+    cache = {}
+    k = 0
+    while True:
+        s = shapes[k % len(shapes)]
+        k += 1
+        if s not in cache:
+            i = by_shape[s][0]
+            cache[s] = tuple(x.astype(np.float64) for x in (inputs.weight_np(w, i), inputs.grad_np(w, step, i),
+                                                              inputs.momentum_np(w, i)))
+        W, g, m = cache[s]
+        t0 = time.perf_counter()
+        oracle.muon_step(W, g, m, lr=w.lr, beta=w.beta, weight_decay=w.weight_decay, nesterov=w.nesterov,
+                         coeffs=coeffs)
+        dt = time.perf_counter() - t0
+        yield dt * 1e3 * total / work(*s), s
+
+
 def run_reference(args, world, rank):
-    """The oracle, as it stands, on the host cores: each step is one bounded sample of the
-    workload (one matrix per shape), scaled to a full step."""
+    """The oracle, as it stands, on the host cores.  Each step is one bounded sample (one
+    matrix, shapes taken in turn) scaled to a full step; value = median over the steps."""
     if rank != 0:
         return
     w = inputs.WORKLOADS[args.workload]
+    gen = oracle_step_samples(w)
     for _ in range(args.warmup):
-        oracle_sample_ms(w)
-    runs = [oracle_sample_ms(w) for _ in range(args.steps)]
-    sample = runs[0][1]
+        next(gen)
+    runs = [next(gen) for _ in range(args.steps)]
     value = statistics.median(r[0] for r in runs)
     cores = blas_threads()
+    sample = (f"per step: the fp64 oracle (momentum, NS x{w.ns_steps}, update) on one matrix of {w.name}, "
+              f"the {len(set(w.shapes))} shapes in turn, scaled to the full step by work ratio; "
+              f"median of {args.steps} steps")
     line = {
         "impl": "reference", "metric": "muon_step_ms", "value": round(value, 3), "unit": "ms",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(value, 3),
@@ -368,27 +418,29 @@ def run_ours(args, world, rank, local):
     launches_per_step = sum(kcount) // prof_steps
 
     # ---- end to end through host buffers: H2D grads, step, D2H params, every step
-    pin_g = torch.empty_like(G, device="cpu").pin_memory()
-    pin_g.copy_(G.cpu())
-    pin_p = torch.empty_like(P, device="cpu").pin_memory()
-    for _ in range(2):
-        G.copy_(pin_g, non_blocking=True)
-        api.muon_step(ps, gs, ms, **kw)
-        pin_p.copy_(P, non_blocking=True)
-    torch.cuda.synchronize()
-    barrier(world)
-    f0 = torch.cuda.Event(enable_timing=True)
-    f1 = torch.cuda.Event(enable_timing=True)
-    e2e_steps = max(1, min(args.steps, 50))
-    f0.record(stream)
-    for _ in range(e2e_steps):
-        G.copy_(pin_g, non_blocking=True)
-        api.muon_step(ps, gs, ms, **kw)
-        pin_p.copy_(P, non_blocking=True)
-    f1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = dist_max(f0.elapsed_time(f1) / e2e_steps, world)
-    barrier(world)
+    e2e_ms = None
+    if not args.no_e2e:
+        pin_g = torch.empty_like(G, device="cpu").pin_memory()
+        pin_g.copy_(G.cpu())
+        pin_p = torch.empty_like(P, device="cpu").pin_memory()
+        for _ in range(2):
+            G.copy_(pin_g, non_blocking=True)
+            api.muon_step(ps, gs, ms, **kw)
+            pin_p.copy_(P, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier(world)
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        e2e_steps = max(1, min(args.steps, 50))
+        f0.record(stream)
+        for _ in range(e2e_steps):
+            G.copy_(pin_g, non_blocking=True)
+            api.muon_step(ps, gs, ms, **kw)
+            pin_p.copy_(P, non_blocking=True)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = dist_max(f0.elapsed_time(f1) / e2e_steps, world)
+        barrier(world)
 
     code, where = api.device_status(ws)
     if code != 0:
@@ -400,26 +452,35 @@ def run_ours(args, world, rank, local):
     peaks, peak_src = load_peaks()
     per_kind = {k: {"ms_total": kms[i], "launches": int(kcount[i])} for i, k in enumerate(KINDS)}
     dom = max(KINDS, key=lambda k: per_kind[k]["ms_total"])
+    # The dominant kernel's work over all its launches in the profiled pass, divided by
+    # their summed time (a workload of several waves has several launches per iteration).
+    iters = {"momentum": 1, "norm": 1, "gram": w.ns_steps, "poly": w.ns_steps, "apply": w.ns_steps - 1,
+             "apply_last": 1}
     dom_launches = max(1, per_kind[dom]["launches"])
     dom_ms = per_kind[dom]["ms_total"] / dom_launches
-    fl = kind_flops(w, dom)
-    by = kind_bytes(w, dom)
+    fl = kind_flops(w, dom) * iters[dom] * prof_steps / dom_launches    # per launch (mean)
+    by = kind_bytes(w, dom) * iters[dom] * prof_steps / dom_launches
     tf = fl / (dom_ms * 1e-3) / 1e12 if fl else 0.0
     gbs = by / (dom_ms * 1e-3) / 1e9
-    f_tensor = tf / peaks["bf16_tflops"] if fl else 0.0
+    # a tensor-bound kernel timed while the power cap held the clocks takes the sustained peak
+    capped = "sw_power_cap" in (clk.get("reasons") or [])
+    tpeak_key = "bf16_tflops_sustained" if capped else "bf16_tflops"
+    f_tensor = tf / peaks[tpeak_key] if fl else 0.0
     f_hbm = gbs / peaks["hbm_gbs"]
     traffic = None
     if NCU_TRAFFIC["source_hash"] == kernel_source_hash() and NCU_TRAFFIC["workload"] == w.name:
         traffic = NCU_TRAFFIC["bytes_per_launch"].get(dom)
     if f_tensor >= f_hbm:
-        roof = {"bound": "tensor", "achieved": round(tf, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+        roof = {"bound": "tensor", "achieved": round(tf, 1), "peak": peaks[tpeak_key], "unit": "TFLOP/s",
                 "frac": round(f_tensor, 4)}
     else:
         roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(f_hbm, 4)}
-    roof.update({"traffic": traffic, "kernel": dom, "peak_source": peak_src,
+    roof.update({"traffic": traffic, "kernel": dom,
+                 "peak_source": peak_src + (" sustained (power cap active)" if capped and roof["bound"] == "tensor"
+                                            else " burst" if roof["bound"] == "tensor" else " copy"),
                  "other_bound_frac": round(min(f_tensor, f_hbm), 4),
-                 "algorithmic_bytes_per_launch": by, "algorithmic_flops_per_launch": fl,
+                 "algorithmic_bytes_per_launch": int(by), "algorithmic_flops_per_launch": int(fl),
                  "ms_per_launch": round(dom_ms, 4)})
 
     alg, dense = step_flops(w)
@@ -435,13 +496,15 @@ def run_ours(args, world, rank, local):
         "ns_tflops": round(world * alg / (ms_step * 1e-3) / 1e12, 1),
         "ns_tflops_dense_equiv": round(world * dense / (ms_step * 1e-3) / 1e12, 1),
         "ns_frac_of_bf16_peak": round(alg / (ms_step * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+        "ns_frac_of_bf16_sustained": round(alg / (ms_step * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"], 4),
         "kernels": {k: {"ms_per_launch": round(v["ms_total"] / max(1, v["launches"]), 4),
                         "launches": v["launches"], "share": round(v["ms_total"] / max(1e-9, sum(
                             x["ms_total"] for x in per_kind.values())), 4)} for k, v in per_kind.items()},
         "roofline": roof,
         "clocks": clk,
-        "e2e": {"value": round(e2e_ms, 4), "unit": "ms", "h2d_bytes_per_step": G.numel() * 4,
-                "d2h_bytes_per_step": P.numel() * P.element_size()},
+        "e2e": None if e2e_ms is None else {
+            "value": round(e2e_ms, 4), "unit": "ms", "h2d_bytes_per_step": G.numel() * 4,
+            "d2h_bytes_per_step": P.numel() * P.element_size()},
         "gpu_launches": int(launches_per_step * args.steps),
         "profiled_steps": prof_steps,
     }
@@ -459,6 +522,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=inputs.WORKLOAD_ORDER)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the host-buffer pass (for workloads whose inputs do not fit pinned host memory)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

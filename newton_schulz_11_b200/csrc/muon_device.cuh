@@ -377,4 +377,19 @@ __device__ __forceinline__ void split_hi_lo(float x, uint32_t& hi, uint32_t& lo)
   lo = float_to_bf16_bits(x - bf16_bits_to_float(hi));
 }
 
+// Two values at once: hi = bf16x2 (x0 in the low half, x1 in the high half) and lo = the
+// bf16x2 of the residuals.  Same roundings as split_hi_lo element by element.
+__device__ __forceinline__ void split_hi_lo2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  const __nv_bfloat162 l =
+      __floats2bfloat162_rn(x0 - __uint_as_float(hi << 16), x1 - __uint_as_float(hi & 0xFFFF0000u));
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// L2 prefetch of the line holding `p`.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 }  // namespace muon

@@ -463,15 +463,17 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
     app[ord_app[k]].tile_begin = tiles_apply;
     tiles_apply += app[ord_app[k]].count * app[ord_app[k]].tiles_per_mat;
   }
-  // The apply runs the staged variant while every Gram side is short: its tiles then
-  // have short reductions, and moving the epilogue's hi/lo by TMA matters more than the
-  // main loop's k-block depth.
+  // The polynomial and the applies run the staged variant while every Gram side is
+  // short: tiles then have short reductions, and moving the epilogue's data by TMA matters
+  // more than the main loop's k-block depth.  Its operand maps have 64 x 64 boxes.  The
+  // Gram, whose epilogue has no inputs, always streams (deeper operand ring).
   int max_m = 0;
   for (const ClassPlan& c : w.classes) max_m = std::max(max_m, static_cast<int>(c.m));
   const bool staged = max_m <= kStagedApplyMaxM;
   for (int cur = 0; cur < 2; ++cur) {
     GemmParams g = base;
     GemmParams a = base;
+    g.staged = 0;
     a.staged = staged ? 1 : 0;
     for (int k = 0; k < nc; ++k) {
       const int ci = ord_sym[k];
@@ -505,12 +507,14 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
     static_cast<GemmParams&>(L->fin[cur]) = a;
   }
   GemmParams pp = base;
+  pp.staged = staged ? 1 : 0;
   for (int k = 0; k < nc; ++k) {
     const int ci = ord_app[k];  // the polynomial's reduction is m, like the apply's
     pp.cls[k] = sym[ci];
     pp.cls[k].ksize = static_cast<int32_t>(w.classes[ci].m);
     pp.cls[k].a_mn = pp.cls[k].b_mn = 0;
-    pp.map_a[k] = pp.map_b[k] = op_a[ci];
+    pp.map_a[k] = pp.map_b[k] = staged ? st_a[ci] : op_a[ci];
+    pp.map_in[k] = st_a[ci];
     pp.map_out[k] = st_b[ci];
   }
   {

@@ -47,20 +47,23 @@
 
 namespace muon {
 
-// Two variants share the kernel.  Streamed (SMALL = false, every mode): 128-deep k-blocks,
-// three 64 KB stages per CTA, a 32 KB epilogue staging area; epilogue inputs are read
-// from global memory.  Staged (SMALL = true, apply modes when the Gram side m is at most
-// 1024): 64-deep k-blocks, three 32 KB stages, and the tile's hi/lo inputs (128 KB per CTA)
-// loaded by TMA into shared memory -- the apply is bound by HBM traffic there, and TMA
-// moves it in full lines.
+// Two variants share the kernel.
+//   Streamed (SMALL = false, for long reductions): 128-deep k-blocks, three 64 KB stages
+//   per CTA, one 32 KB epilogue staging area; epilogue inputs are read from global memory.
+//   Staged (SMALL = true, when every Gram side m of the launch is at most 1024): 64-deep
+//   k-blocks in 32 KB stages, and the epilogue's inputs moved by TMA through shared
+//   memory -- there tiles are short, and the epilogue, not the main loop, sets the pace.
+//     Gram        five stages; two 32 KB output staging buffers (stores of one quarter
+//                 drain while the next is written)
+//     polynomial  three stages; two output buffers; the tile's A block (64 KB) staged
+//     apply       three stages; the tile's hi and lo (128 KB) staged and updated in place
 template <int MODE, bool SMALL = false>
 struct Lay {
   static constexpr bool kSym = MODE == kGram || MODE == kPoly;
-  static_assert(!(SMALL && kSym), "the staged variant is an apply");
   static constexpr int TM = 256;  // pair tile rows (128 per CTA)
   static constexpr int TN = 256;  // pair tile columns = UMMA N
   static constexpr int BK = SMALL ? 64 : 128;
-  static constexpr int S = 3;
+  static constexpr int S = (SMALL && MODE == kGram) ? 5 : 3;
   static constexpr int NEPI = 8;
   static constexpr int kBox64 = 64 * 64 * 2;       // one 64 x 64 box: 8 KB
   static constexpr int kHalf = kBM * kBox * 2;      // one 64 x 128 box: 16 KB
@@ -69,8 +72,8 @@ struct Lay {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kRing = S * kStageBytes;
   // streamed: one 64-column quarter of this CTA's 128 x 256 tile at a time (symmetric
-  // modes D_q and T_q, apply hi_q and lo_q); staged: the tile's hi and lo, 128 x 256 each
-  static constexpr int kEpi = SMALL ? 8 * kHalf : 2 * kHalf;
+  // modes D_q and T_q, apply hi_q and lo_q); staged: see above
+  static constexpr int kEpi = !SMALL ? 2 * kHalf : (MODE == kGram ? 4 * kHalf : 8 * kHalf);
   static constexpr int kBarOff = kRing + kEpi;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;
   static constexpr int kEpiThreads = 32 * NEPI;
@@ -199,13 +202,12 @@ __device__ __forceinline__ void store_region(const CUtensorMap* map, const uint8
       tma_store_3d(map, buf + ((4 * rb + cb) << 13), col0 + 64 * cb, row0 + 64 * rb, mat);
 }
 
-__device__ __forceinline__ void load_region(uint8_t* buf, const CUtensorMap* map, uint64_t* bar, int row0, int col0,
-                                            int mat) {
+// Loads column box cb (both row boxes) of the staged region.
+__device__ __forceinline__ void load_region_quarter(uint8_t* buf, const CUtensorMap* map, uint64_t* bar, int cb,
+                                                    int row0, int col0, int mat) {
 #pragma unroll
   for (int rb = 0; rb < 2; ++rb)
-#pragma unroll
-    for (int cb = 0; cb < 4; ++cb)
-      tma_load_3d(buf + ((4 * rb + cb) << 13), map, bar, col0 + 64 * cb, row0 + 64 * rb, mat);
+    tma_load_3d(buf + ((4 * rb + cb) << 13), map, bar, col0 + 64 * cb, row0 + 64 * rb, mat);
 }
 
 __device__ __forceinline__ uint4 pack8(const uint32_t* b) {
@@ -388,13 +390,7 @@ __device__ __forceinline__ void apply_quarter(const typename ParamsOf<MODE>::typ
   }
   if constexpr (MODE == kApply) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      uint32_t h0, l0, h1, l1;
-      split_hi_lo(x[2 * i], h0, l0);
-      split_hi_lo(x[2 * i + 1], h1, l1);
-      hb[i] = h0 | (h1 << 16);
-      lb[i] = l0 | (l1 << 16);
-    }
+    for (int i = 0; i < 16; ++i) split_hi_lo2(x[2 * i], x[2 * i + 1], hb[i], lb[i]);
   } else {
     (void)hb;
     (void)lb;
@@ -423,19 +419,17 @@ __device__ __forceinline__ void apply_staged(const typename ParamsOf<MODE>::type
   float x[32];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    x[2 * i] = s * fmaf(p.a, lo_bf16(xh[i]) + lo_bf16(xl[i]), __uint_as_float(v[2 * i]));
-    x[2 * i + 1] = s * fmaf(p.a, hi_bf16(xh[i]) + hi_bf16(xl[i]), __uint_as_float(v[2 * i + 1]));
+    x[2 * i] = fmaf(p.a, lo_bf16(xh[i]) + lo_bf16(xl[i]), __uint_as_float(v[2 * i]));
+    x[2 * i + 1] = fmaf(p.a, hi_bf16(xh[i]) + hi_bf16(xl[i]), __uint_as_float(v[2 * i + 1]));
+  }
+  if (s != 1.f) {  // iteration 0 only (uniform)
+#pragma unroll
+    for (int j = 0; j < 32; ++j) x[j] *= s;
   }
   if constexpr (MODE == kApply) {
     uint32_t hb[16], lb[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      uint32_t h0, l0, h1, l1;
-      split_hi_lo(x[2 * i], h0, l0);
-      split_hi_lo(x[2 * i + 1], h1, l1);
-      hb[i] = h0 | (h1 << 16);
-      lb[i] = l0 | (l1 << 16);
-    }
+    for (int i = 0; i < 16; ++i) split_hi_lo2(x[2 * i], x[2 * i + 1], hb[i], lb[i]);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const uint32_t o = region_chunk(r, (c0 >> 3) + q);
@@ -464,8 +458,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + 2;  // used in the leader CTA: both CTAs' epilogues arrive
   uint64_t* tdown = tempty + 2;
-  uint64_t* efull = tdown + 1;  // staged variant: the tile's hi/lo inputs have landed
-  uint64_t* pdone = efull + 1;  // used in the leader CTA: the peer's producer has finished
+  uint64_t* efull = tdown + 1;  // staged variant: quarter q of the tile's hi/lo inputs has landed
+  uint64_t* pdone = efull + 4;  // used in the leader CTA: the peer's producer has finished
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pdone + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* epi_flag = abort_flag + 1;
@@ -489,7 +483,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
       mbar_init(&tempty[a], 2 * L::NEPI);
     }
     mbar_init(tdown, 1);
-    mbar_init(efull, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(&efull[q], 1);
     mbar_init(pdone, 1);
     *abort_flag = 0;
     *epi_flag = 0;
@@ -641,79 +635,120 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
       }
       quiet_wait(tdown, 0, tb);
     }
-  } else if constexpr (SMALL) {
+  } else if constexpr (SMALL && !kSym) {
     // ---------------------------------------------------------------- staged apply epilogue (both CTAs)
-    // The tile's old hi/lo (128 x 256 each per CTA) are loaded by TMA into the staging
-    // region by the epilogue leader as soon as the previous tile is done with it, so they
-    // are in place before the accumulator is; kApply updates them in place and stores
-    // them back by TMA, one 128-column half at a time.
+    // The tile's old hi/lo (128 x 256 each per CTA) live in the staging region as four
+    // 64-column quarters, each with its own barrier.  Quarter q is updated (kApply: in
+    // place, then stored by TMA) and, as soon as nothing reads it any more, refilled with
+    // quarter q of this pair's next tile, so the loads run three quarters ahead of use.
     const int ew = warp - 2;
     const int q4 = warp & 3;  // TMEM lanes 32 q4 .. 32 q4 + 31 belong to this warp
-    const int h = ew >> 2;    // which 64 columns of each 128-column half
+    const int h = ew >> 2;    // which 32 columns of each quarter
     const int r = q4 * 32 + lane;
-    const bool leader = threadIdx.x == 64;
+    const bool leader = threadIdx.x == 64;  // also the thread that waits on the barriers
     const uint32_t tempty0 = map_to_rank(smem_u32(tempty), 0);
     uint8_t* hib = epi;
     uint8_t* lob = epi + 4 * L::kHalf;
     int acc = 0;
     uint32_t aph = 0;
-    bool in_pending = false;  // leader: a load into the region has not been waited for
-    uint32_t in_par = 0;
-    auto load_inputs = [&](int tt, uint32_t par) {
-      const Tile nx = decode_tile<MODE>(p, tt);
+    uint32_t pending = 0, pend_par = 0;  // leader: quarter loads not yet waited for, and their parity
+    auto load_quarter = [&](const Tile& nx, int q, uint32_t par) {
       const int row0 = L::TM * nx.I + kBM * rank, col0 = L::TN * nx.J;
-      mbar_arrive_expect_tx(efull, 8 * L::kHalf);
-      load_region(hib, &p.map_in[nx.cls], efull, row0, col0, nx.mat);
-      load_region(lob, &p.map_out2[nx.cls], efull, row0, col0, nx.mat);
-      in_pending = true;
-      in_par = par;
+      mbar_arrive_expect_tx(&efull[q], 2 * L::kHalf);
+      load_region_quarter(hib, &p.map_in[nx.cls], &efull[q], q, row0, col0, nx.mat);
+      load_region_quarter(lob, &p.map_out2[nx.cls], &efull[q], q, row0, col0, nx.mat);
+      pending |= 1u << q;
+      pend_par = (pend_par & ~(1u << q)) | (par << q);
     };
-    if (leader && pair < p.total_tiles) load_inputs(pair, 0u);
+    if (leader && pair < p.total_tiles) {
+      const Tile first = decode_tile<MODE>(p, pair);
+      for (int q = 0; q < 4; ++q) load_quarter(first, q, 0u);
+    }
     int k = 0;
-    for (int t = pair; t < p.total_tiles; t += npairs, ++k) {
+    bool live = true;
+    for (int t = pair; live && t < p.total_tiles; t += npairs, ++k) {
       const Tile tl = decode_tile<MODE>(p, t);
       const ClassDesc& cd = p.cls[tl.cls];
       const uint32_t kpar = static_cast<uint32_t>(k) & 1u;
-      if (ew == 0) {
-        bool ok = warp_wait(&tfull[acc], aph, wd, kSiteEpilogueFull);
-        if (ok) ok = warp_wait(efull, kpar, wd, kSiteEpilogueIn);
-        if (lane == 0) *epi_flag = ok ? 1 : 0;
-      }
-      named_barrier(1, NT);
-      if (*epi_flag == 0) break;
-      in_pending = false;
-      tc_fence_after();
-      const uint32_t tacc = tmem_base + static_cast<uint32_t>(acc * L::TN) + (static_cast<uint32_t>(q4 * 32) << 16);
+      const bool has_next = t + npairs < p.total_tiles;
+      Tile nx = tl;
+      if (has_next) nx = decode_tile<MODE>(p, t + npairs);
       const float sc = p.first_iter ? p.scale[cd.mat_base + tl.mat] : 1.f;
       const int row0 = L::TM * tl.I + kBM * rank, col0 = L::TN * tl.J;
+      const uint32_t tacc = tmem_base + static_cast<uint32_t>(acc * L::TN) + (static_cast<uint32_t>(q4 * 32) << 16);
 #pragma unroll 1
-      for (int hh = 0; hh < 2; ++hh) {
-        const int c0 = 128 * hh + 64 * h;
+      for (int q = 0; q < 4; ++q) {
+        // One warp waits (for the accumulator first, then for the inputs: kApply one
+        // quarter at a time, kApplyLast all four at once); the rest learn the outcome at
+        // the barrier, so every epilogue warp leaves together.
+        if (MODE == kApply || q == 0) {
+          if (ew == 0) {
+            bool ok = q > 0 || warp_wait(&tfull[acc], aph, wd, kSiteEpilogueFull);
+            const int q_hi = MODE == kApply ? q : 3;
+            for (int qq = q; ok && qq <= q_hi; ++qq) ok = warp_wait(&efull[qq], kpar, wd, kSiteEpilogueIn);
+            if (lane == 0) {
+              *epi_flag = ok ? 1 : 0;
+              if (ok) pending &= ~(((2u << q_hi) - 1u) & ~((1u << q) - 1u));
+            }
+          }
+          named_barrier(1, NT);
+          if (*epi_flag == 0) {
+            live = false;
+            break;
+          }
+        }
+        if (q == 0) {
+          tc_fence_after();
+          if constexpr (MODE == kApplyLast) {
+            // warm L2 with this thread's row of W in the next tile
+            if (has_next) {
+              const ClassDesc& nd = p.cls[nx.cls];
+              const UpdMat& un = p.upd[nd.mat_base + nx.mat];
+              const int Rn = L::TM * nx.I + kBM * rank + r, Cn = L::TN * nx.J;
+              if (un.param != nullptr && Rn < nd.rows) {
+                const int esz = un.param_bf16 ? 2 : 4;
+                const int bytes = (nd.cols - Cn < L::TN ? nd.cols - Cn : L::TN) * esz;
+                const char* row = static_cast<const char*>(un.param) + (static_cast<int64_t>(Rn) * un.ld_param + Cn) * esz;
+                for (int off = 0; off < bytes; off += 128) prefetch_l2(row + off);
+                prefetch_l2(row + bytes - 1);
+              }
+            }
+          }
+        }
+        const int c0 = 64 * q + 32 * h;
         apply_staged<MODE>(p, cd, tl, rank, r, c0, tacc + c0, hib, lob, sc);
-        apply_staged<MODE>(p, cd, tl, rank, r, c0 + 32, tacc + c0 + 32, hib, lob, sc);
-        if (hh == 1) {
+        if (q == 3) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * static_cast<uint32_t>(acc));
         }
         if constexpr (MODE == kApply) {
           fence_proxy_async_smem();
-          named_barrier(1, NT);
+          named_barrier(1, NT);  // quarter q is final
           if (leader) {
-            store_region(&p.map_out[tl.cls], hib, 2 * hh, 2, row0, col0, tl.mat);
-            store_region(&p.map_out2[tl.cls], lob, 2 * hh, 2, row0, col0, tl.mat);
+            store_region(&p.map_out[tl.cls], hib, q, 1, row0, col0, tl.mat);
+            store_region(&p.map_out2[tl.cls], lob, q, 1, row0, col0, tl.mat);
             bulk_commit();
+            // the stores of quarter q - 1 have read their boxes: refill them
+            if (q > 0) {
+              bulk_wait_read<1>();
+              if (has_next) load_quarter(nx, q - 1, kpar ^ 1u);
+            }
           }
         }
       }
-      // the region is refilled once nothing reads it any more
+      if (!live) break;
       if constexpr (MODE == kApply) {
-        if (leader) bulk_wait_read<0>();
+        if (leader) {
+          bulk_wait_read<0>();
+          if (has_next) load_quarter(nx, 3, kpar ^ 1u);
+        }
       } else {
         fence_proxy_async_smem();
-        named_barrier(1, NT);
+        named_barrier(1, NT);  // nothing reads the region any more
+        if (leader && has_next)
+          for (int q = 0; q < 4; ++q) load_quarter(nx, q, kpar ^ 1u);
       }
-      if (leader && t + npairs < p.total_tiles) load_inputs(t + npairs, kpar ^ 1u);
       if (++acc == 2) {
         acc = 0;
         aph ^= 1u;
@@ -721,7 +756,106 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
     }
     if (leader) {
       bulk_wait_all();
-      if (in_pending) quiet_wait(efull, in_par, tb);
+      for (int q = 0; q < 4; ++q)
+        if (pending & (1u << q)) quiet_wait(&efull[q], (pend_par >> q) & 1u, tb);
+    }
+  } else if constexpr (SMALL) {
+    // ---------------------------------------------------------------- staged symmetric epilogue (both CTAs)
+    // Output quarters alternate between two staging buffers, so the TMA stores of one
+    // drain while the next is written.  The polynomial's A block is staged like the
+    // apply's inputs: four 64-column quarters, each refilled for the next tile as soon as
+    // it has been read.
+    const int ew = warp - 2;
+    const int q4 = warp & 3;
+    const int h = ew >> 2;
+    const int r = q4 * 32 + lane;
+    const bool leader = threadIdx.x == 64;  // also the thread that waits on the barriers
+    const uint32_t tempty0 = map_to_rank(smem_u32(tempty), 0);
+    uint8_t* Ain = epi + 4 * L::kHalf;
+    int acc = 0;
+    uint32_t aph = 0;
+    uint32_t pending = 0, pend_par = 0;
+    uint32_t used = 0;  // output quarters handed to TMA stores so far (uniform)
+    auto load_quarter = [&](const Tile& nx, int q, uint32_t par) {
+      mbar_arrive_expect_tx(&efull[q], L::kHalf);
+      load_region_quarter(Ain, &p.map_in[nx.cls], &efull[q], q, L::TM * nx.I + kBM * rank, L::TN * nx.J, nx.mat);
+      pending |= 1u << q;
+      pend_par = (pend_par & ~(1u << q)) | (par << q);
+    };
+    if (MODE == kPoly && leader && pair < p.total_tiles) {
+      const Tile first = decode_tile<MODE>(p, pair);
+      for (int q = 0; q < 4; ++q) load_quarter(first, q, 0u);
+    }
+    int k = 0;
+    bool live = true;
+    for (int t = pair; live && t < p.total_tiles; t += npairs, ++k) {
+      const Tile tl = decode_tile<MODE>(p, t);
+      const ClassDesc& cd = p.cls[tl.cls];
+      const uint32_t kpar = static_cast<uint32_t>(k) & 1u;
+      const bool has_next = t + npairs < p.total_tiles;
+      Tile nx = tl;
+      if (has_next) nx = decode_tile<MODE>(p, t + npairs);
+      const int rb = 2 * tl.I + rank;
+      float mul = 1.f;
+      if (MODE == kGram && p.first_iter) {
+        const float sv = p.scale[cd.mat_base + tl.mat];
+        mul = sv * sv;
+      }
+      const uint32_t tacc = tmem_base + static_cast<uint32_t>(acc * L::TN) + (static_cast<uint32_t>(q4 * 32) << 16);
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        const int cb = 2 * tl.J + (q >> 1);
+        const bool skip = rb > cb;  // below the diagonal: stored by the block's mirror (uniform)
+        if (ew == 0) {
+          bool ok = q > 0 || warp_wait(&tfull[acc], aph, wd, kSiteEpilogueFull);
+          if (MODE == kPoly && ok) ok = warp_wait(&efull[q], kpar, wd, kSiteEpilogueIn);
+          if (lane == 0) {
+            *epi_flag = ok ? 1 : 0;
+            if (ok) pending &= ~(1u << q);
+            if (!skip) bulk_wait_read<1>();  // the stores that used this buffer last have read it
+          }
+        }
+        named_barrier(1, NT);
+        if (*epi_flag == 0) {
+          live = false;
+          break;
+        }
+        if (q == 0) tc_fence_after();
+        if (!skip) {
+          uint8_t* Q = epi + (used & 1u) * (2 * L::kHalf);
+          uint8_t* Tst = Q + L::kHalf;
+          uint4 ain[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            ain[i] = MODE == kPoly ? *reinterpret_cast<const uint4*>(Ain + region_chunk(r, 8 * q + 4 * h + i))
+                                   : make_uint4(0u, 0u, 0u, 0u);
+          sym_quarter<MODE>(p, mul, rb == cb, r, h, tacc + 64 * q + 32 * h, Q, Tst, ain);
+          fence_proxy_async_smem();
+          named_barrier(1, NT);
+          if (leader) {
+            store_q(&p.map_out[tl.cls], Q, kBM * rb, kBM * cb + 64 * (q & 1), tl.mat);
+            if (rb != cb) store_t(&p.map_out[tl.cls], Tst, kBM * cb + 64 * (q & 1), kBM * rb, tl.mat);
+            bulk_commit();
+          }
+          ++used;
+        }
+        if (q == 3) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * static_cast<uint32_t>(acc));
+        }
+        if (MODE == kPoly && leader && has_next) load_quarter(nx, q, kpar ^ 1u);
+      }
+      if (!live) break;
+      if (++acc == 2) {
+        acc = 0;
+        aph ^= 1u;
+      }
+    }
+    if (leader) {
+      bulk_wait_all();
+      for (int q = 0; q < 4; ++q)
+        if (pending & (1u << q)) quiet_wait(&efull[q], (pend_par >> q) & 1u, tb);
     }
   } else {
     // ---------------------------------------------------------------- epilogue (both CTAs)
@@ -919,8 +1053,10 @@ int gemm_tile_cols() { return 256; }
 // p->staged set run the staged variant, whose operand maps have 64 x 64 boxes.
 cudaError_t launch_gemm(int mode, const GemmParams* p, int max_pairs, cudaStream_t stream) {
   switch (mode) {
-    case kGram: return launch_one<kGram, false>(*p, max_pairs, stream);
-    case kPoly: return launch_one<kPoly, false>(*p, max_pairs, stream);
+    case kGram:
+      return p->staged ? launch_one<kGram, true>(*p, max_pairs, stream) : launch_one<kGram, false>(*p, max_pairs, stream);
+    case kPoly:
+      return p->staged ? launch_one<kPoly, true>(*p, max_pairs, stream) : launch_one<kPoly, false>(*p, max_pairs, stream);
     case kApply:
       return p->staged ? launch_one<kApply, true>(*p, max_pairs, stream)
                        : launch_one<kApply, false>(*p, max_pairs, stream);
