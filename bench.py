@@ -275,6 +275,14 @@ def barrier(world):
 
 # ------------------------------------------------------------------ reference arm
 
+def workload_of(args):
+    w = inputs.WORKLOADS[args.workload]
+    k = getattr(args, "matrices", 0)
+    if k and k < len(w.shapes):
+        w = inputs.scaled_workload(w, w.shapes[:k], name=f"{w.name}[:{k}]")
+    return w
+
+
 def oracle_step_samples(w):
     """One bounded sample per reference step: the fp64 oracle's step on ONE matrix,
     cycling through the workload's distinct shapes; each sample is scaled to a full step
@@ -318,7 +326,7 @@ def run_reference(args, world, rank):
     matrix, shapes taken in turn) scaled to a full step; value = median over the steps."""
     if rank != 0:
         return
-    w = inputs.WORKLOADS[args.workload]
+    w = workload_of(args)
     gen = oracle_step_samples(w)
     for _ in range(args.warmup):
         next(gen)
@@ -351,7 +359,7 @@ def run_ours(args, world, rank, local):
     build.build()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    w = inputs.WORKLOADS[args.workload]
+    w = workload_of(args)
     coeffs = load_coeffs(w)
     step0 = inputs.first_step_index(w)
 
@@ -525,6 +533,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer pass (for workloads whose inputs do not fit pinned host memory)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--matrices", type=int, default=0,
+                    help="run only the first K matrices of the workload (a small case of the same kernels)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

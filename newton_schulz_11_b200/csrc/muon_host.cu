@@ -465,8 +465,9 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
   }
   // The polynomial and the applies run the staged variant while every Gram side is
   // short: tiles then have short reductions, and moving the epilogue's data by TMA matters
-  // more than the main loop's k-block depth.  Its operand maps have 64 x 64 boxes.  The
-  // Gram, whose epilogue has no inputs, always streams (deeper operand ring).
+  // more than the main loop's k-block depth.  There K-major operands load 64 x 128 boxes
+  // (one per 64-deep k-block) and MN-major ones 64 x 64 boxes.  The Gram, whose epilogue
+  // has no inputs, always streams (deeper operand ring).
   int max_m = 0;
   for (const ClassPlan& c : w.classes) max_m = std::max(max_m, static_cast<int>(c.m));
   const bool staged = max_m <= kStagedApplyMaxM;
@@ -487,8 +488,10 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
       a.cls[k] = app[cj];
       a.cls[k].x_hi_cur = reinterpret_cast<__nv_bfloat16*>(ws + w.classes[cj].off_hi[cur]);
       a.cls[k].x_hi_next = reinterpret_cast<__nv_bfloat16*>(ws + w.classes[cj].off_hi[cur ^ 1]);
-      const CUtensorMap& x_op = staged ? st_hi[cj][cur] : op_hi[cj][cur];
-      const CUtensorMap& b_op = staged ? st_b[cj] : op_b[cj];
+      // staged: K-major operands load 128-row boxes, MN-major ones 64 x 64 boxes
+      const bool x_mn = !w.classes[cj].tall;  // wide: X is the MN-major B operand
+      const CUtensorMap& x_op = (staged && x_mn) ? st_hi[cj][cur] : op_hi[cj][cur];
+      const CUtensorMap& b_op = op_b[cj];
       if (w.classes[cj].tall) {
         a.map_a[k] = x_op;
         a.map_b[k] = b_op;
@@ -513,7 +516,7 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
     pp.cls[k] = sym[ci];
     pp.cls[k].ksize = static_cast<int32_t>(w.classes[ci].m);
     pp.cls[k].a_mn = pp.cls[k].b_mn = 0;
-    pp.map_a[k] = pp.map_b[k] = staged ? st_a[ci] : op_a[ci];
+    pp.map_a[k] = pp.map_b[k] = op_a[ci];
     pp.map_in[k] = st_a[ci];
     pp.map_out[k] = st_b[ci];
   }

@@ -146,21 +146,25 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t) {
   return r;
 }
 
-// Half i of an operand tile (128 MN x BK), completing on the leader CTA's mbarrier.
-//   BK = 128 (64 x 128 boxes): K-major -> K columns [k0 + 64 i, +64) of 128 rows;
-//                              MN-major -> MN columns [mn0 + 64 i, +64) of 128 K-rows.
-//   BK = 64 (64 x 64 boxes):   K-major -> rows [mn0 + 64 i, +64) of 64 K columns;
-//                              MN-major -> MN columns [mn0 + 64 i, +64) of 64 K-rows.
-// In both cases half i lands at i x (its bytes), which is the layout operand_desc reads.
+// One operand tile (128 MN x BK) into `dst`, completing on the leader CTA's mbarrier.
+//   BK = 128 (64 x 128 boxes): K-major -> two boxes, K columns [k0 + 64 i, +64) of 128 rows;
+//                              MN-major -> two boxes, MN columns [mn0 + 64 i, +64) of 128 K-rows.
+//   BK = 64: K-major (64 x 128 box) -> one box, 64 K columns of 128 rows;
+//            MN-major (64 x 64 boxes) -> two boxes, MN columns [mn0 + 64 i, +64) of 64 K-rows.
+// Box i lands at i x (its bytes), which is the layout operand_desc reads.
 template <int BK>
-__device__ __forceinline__ void load_half_pair(void* dst, const CUtensorMap* map, int mn_major, int mn0, int k0,
-                                               int i, int mat, uint32_t bar_cluster) {
-  if (mn_major)
-    tma_load_3d_pair(dst, map, bar_cluster, mn0 + 64 * i, k0, mat);
-  else if (BK == 128)
-    tma_load_3d_pair(dst, map, bar_cluster, k0 + 64 * i, mn0, mat);
-  else
-    tma_load_3d_pair(dst, map, bar_cluster, k0, mn0 + 64 * i, mat);
+__device__ __forceinline__ void load_operand_pair(uint8_t* dst, const CUtensorMap* map, int mn_major, int mn0, int k0,
+                                                  int mat, uint32_t bar_cluster) {
+  constexpr int kBoxBytes = kBM * BK;  // half of the tile's bytes
+  if (mn_major) {
+    tma_load_3d_pair(dst, map, bar_cluster, mn0, k0, mat);
+    tma_load_3d_pair(dst + kBoxBytes, map, bar_cluster, mn0 + 64, k0, mat);
+  } else if (BK == 128) {
+    tma_load_3d_pair(dst, map, bar_cluster, k0, mn0, mat);
+    tma_load_3d_pair(dst + kBoxBytes, map, bar_cluster, k0 + 64, mn0, mat);
+  } else {
+    tma_load_3d_pair(dst, map, bar_cluster, k0, mn0, mat);
+  }
 }
 
 // Shared-memory descriptor of the kk-th 16-deep K slice (kk < BK / 16) of a staged operand:
@@ -308,7 +312,7 @@ __device__ __forceinline__ void sym_quarter(const GemmParams& p, float mul, bool
 // columns [c0, c0 + 32) of this CTA's tile row r;  O <- x  and/or  W <- W decay - lr_scale x.
 template <int MODE>
 __device__ __forceinline__ void write_update(const FinalParams& p, const ClassDesc& cd, const Tile& tl, int rank,
-                                             int r, int c0, const float (&x)[32]) {
+                                             int r, int c0, const float (&x)[32], const uint4* w_pre = nullptr) {
   const int R = Lay<MODE>::TM * tl.I + kBM * rank + r;
   const int C0 = Lay<MODE>::TN * tl.J + c0;
   const int cols = cd.cols;
@@ -334,7 +338,7 @@ __device__ __forceinline__ void write_update(const FinalParams& p, const ClassDe
       if (full && u.vec_param) {
         uint4 raw[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) raw[q] = reinterpret_cast<const uint4*>(w)[q];
+        for (int q = 0; q < 4; ++q) raw[q] = w_pre != nullptr ? w_pre[q] : reinterpret_cast<const uint4*>(w)[q];
         const uint32_t* rw = reinterpret_cast<const uint32_t*>(raw);
         uint32_t wb[16];
 #pragma unroll
@@ -369,6 +373,22 @@ __device__ __forceinline__ void write_update(const FinalParams& p, const ClassDe
   }
 }
 
+// The bf16 W row segment write_update reads for tile columns [c0, c0 + 32) of this CTA's
+// tile row r, loaded ahead of time; false where write_update takes another path.
+template <int MODE>
+__device__ __forceinline__ bool load_w_segment(const FinalParams& p, const ClassDesc& cd, const Tile& tl, int rank,
+                                               int r, int c0, uint4 (&w)[4]) {
+  const UpdMat& u = p.upd[cd.mat_base + tl.mat];
+  const int R = Lay<MODE>::TM * tl.I + kBM * rank + r;
+  const int C0 = Lay<MODE>::TN * tl.J + c0;
+  if (u.param == nullptr || !u.param_bf16 || !u.vec_param || R >= cd.rows || C0 + 32 > cd.cols) return false;
+  const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(u.param) +
+                                                    static_cast<int64_t>(R) * u.ld_param + C0);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) w[q] = src[q];
+  return true;
+}
+
 // X update for the 32 tile columns [c0, c0 + 32) of this CTA's tile row r, with the old
 // hi/lo pair already in registers: x = s (a (hi + lo) + acc).  kApply returns the new
 // pair packed (hb, lb); kApplyLast updates W and/or writes O in global memory.
@@ -398,12 +418,13 @@ __device__ __forceinline__ void apply_quarter(const typename ParamsOf<MODE>::typ
   }
 }
 
-// Staged variant of the same update: the old pair is read from the staged region, and
-// kApply writes the new pair back in place (the region is then stored by TMA).
+// Staged variant of the same update: the old pair is read from the staged region; kApply
+// writes the new pair back in place (the region is then stored by TMA), kApplyLast updates
+// W and/or writes O (w_pre: this thread's W segment, loaded ahead, or nullptr).
 template <int MODE>
 __device__ __forceinline__ void apply_staged(const typename ParamsOf<MODE>::type& p, const ClassDesc& cd,
                                              const Tile& tl, int rank, int r, int c0, uint32_t tcol, uint8_t* hib,
-                                             uint8_t* lob, float s) {
+                                             uint8_t* lob, float s, const uint4* w_pre = nullptr) {
   uint32_t v[32];
   tmem_ld_32x32b_x32(tcol, v);
   uint4 xh4[4], xl4[4];
@@ -437,7 +458,7 @@ __device__ __forceinline__ void apply_staged(const typename ParamsOf<MODE>::type
       *reinterpret_cast<uint4*>(lob + o) = make_uint4(lb[4 * q], lb[4 * q + 1], lb[4 * q + 2], lb[4 * q + 3]);
     }
   } else {
-    write_update<MODE>(p, cd, tl, rank, r, c0, x);
+    write_update<MODE>(p, cd, tl, rank, r, c0, x, w_pre);
   }
 }
 
@@ -542,11 +563,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
           if (leader_cta) mbar_arrive_expect_tx(&full[s], 2 * L::kStageBytes);
           const uint32_t fb = full0 + 8u * static_cast<uint32_t>(s);
           const int k0 = kb * L::BK;
-          constexpr int kPart = L::kABytes / 2;
-          load_half_pair<L::BK>(sa, ma, cd.a_mn, a0, k0, 0, tl.mat, fb);
-          load_half_pair<L::BK>(sa + kPart, ma, cd.a_mn, a0, k0, 1, tl.mat, fb);
-          load_half_pair<L::BK>(sb, mb, cd.b_mn, b0, k0, 0, tl.mat, fb);
-          load_half_pair<L::BK>(sb + kPart, mb, cd.b_mn, b0, k0, 1, tl.mat, fb);
+          load_operand_pair<L::BK>(sa, ma, cd.a_mn, a0, k0, tl.mat, fb);
+          load_operand_pair<L::BK>(sb, mb, cd.b_mn, b0, k0, tl.mat, fb);
           ++issued;
           if (++s == S) {
             s = 0;
@@ -676,6 +694,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
       const float sc = p.first_iter ? p.scale[cd.mat_base + tl.mat] : 1.f;
       const int row0 = L::TM * tl.I + kBM * rank, col0 = L::TN * tl.J;
       const uint32_t tacc = tmem_base + static_cast<uint32_t>(acc * L::TN) + (static_cast<uint32_t>(q4 * 32) << 16);
+      // kApplyLast: this thread's bf16 W segment for the quarter after the one being
+      // computed is loaded one quarter ahead (the first before the accumulator wait)
+      uint4 wq[4];
+      bool wq_ok = false;
+      if constexpr (MODE == kApplyLast) wq_ok = load_w_segment<MODE>(p, cd, tl, rank, r, 32 * h, wq);
 #pragma unroll 1
       for (int q = 0; q < 4; ++q) {
         // One warp waits (for the accumulator first, then for the inputs: kApply one
@@ -716,7 +739,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
           }
         }
         const int c0 = 64 * q + 32 * h;
-        apply_staged<MODE>(p, cd, tl, rank, r, c0, tacc + c0, hib, lob, sc);
+        if constexpr (MODE == kApplyLast) {
+          uint4 wn[4];
+          const bool wn_ok = q < 3 && load_w_segment<MODE>(p, cd, tl, rank, r, c0 + 64, wn);
+          apply_staged<MODE>(p, cd, tl, rank, r, c0, tacc + c0, hib, lob, sc, wq_ok ? wq : nullptr);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) wq[i] = wn[i];
+          wq_ok = wn_ok;
+        } else {
+          apply_staged<MODE>(p, cd, tl, rank, r, c0, tacc + c0, hib, lob, sc);
+        }
         if (q == 3) {
           tc_fence_before();
           __syncwarp();
