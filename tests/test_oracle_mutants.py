@@ -127,3 +127,89 @@ def test_unmutated_oracle_passes_every_detector():
 def test_planted_mistake_is_caught(monkeypatch, name, mutant, detector):
     monkeypatch.setattr(mo, name, mutant)
     assert detector(), f"mutant {mutant.__name__} of {name} slipped through the pins"
+
+
+# ------------------------------------------------------------------ AdamW oracle
+
+import oracle.adamw_oracle as ao  # noqa: E402
+
+
+def _adamw_pins_fail():
+    h = load_golden("adamw_handworked.json")
+    m = np.zeros(3)
+    v = np.zeros(3)
+    for g, m_exp, v_exp in zip(h["grads"], h["m"], h["v"]):
+        m, v = ao.adamw_moments(m, v, np.array(g), h["beta1"], h["beta2"])
+        if not (np.array_equal(m, np.array(m_exp)) and np.array_equal(v, np.array(v_exp))):
+            return True
+    f = h["first_step"]
+    p1, _, _ = ao.adamw_step(np.array(f["p0"]), np.array(h["grads"][0]), np.zeros(3), np.zeros(3), lr=f["lr"],
+                             beta1=h["beta1"], beta2=h["beta2"], eps=f["eps"], weight_decay=f["weight_decay"],
+                             step=1)
+    if not np.allclose(p1, f["p1"], rtol=0, atol=1e-15):
+        return True
+    g = np.array([0.3, -2.0, 1e-3, 5.0])
+    p = np.zeros(4)
+    m = np.zeros(4)
+    v = np.zeros(4)
+    for t in range(1, 6):
+        p_new, m, v = ao.adamw_step(p, g, m, v, lr=0.01, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, step=t)
+        if not np.allclose(p - p_new, 0.01 * g / (np.abs(g) + 1e-8), rtol=1e-12, atol=0):
+            return True
+        p = p_new
+    p0 = np.array([1.0, -3.0, 0.5])
+    p, _, _ = ao.adamw_step(p0, np.zeros(3), np.zeros(3), np.zeros(3), lr=0.1, beta1=0.9, beta2=0.999, eps=1e-8,
+                            weight_decay=0.5, step=1)
+    if not np.allclose(p, 0.95 * p0, rtol=1e-15, atol=0):
+        return True
+    _, m, v = ao.adamw_step(np.zeros(1), np.array([1e-12]), np.zeros(1), np.zeros(1), lr=1.0, beta1=0.9,
+                            beta2=0.999, eps=1e-8, weight_decay=0.0, step=1)
+    return not np.allclose(ao.adamw_direction(m, v, 0.9, 0.999, 1e-8, 1), 1e-12 / (1e-12 + 1e-8), rtol=1e-12)
+
+
+def _mut_adam_swapped_betas(m, v, g, beta1, beta2):
+    g = np.asarray(g, np.float64)
+    return beta2 * m + (1 - beta2) * g, beta1 * v + (1 - beta1) * g * g
+
+
+def _mut_adam_abs_second_moment(m, v, g, beta1, beta2):
+    g = np.asarray(g, np.float64)
+    return beta1 * m + (1 - beta1) * g, beta2 * v + (1 - beta2) * np.abs(g)
+
+
+def _mut_adam_no_bias_correction(m, v, beta1, beta2, eps, step):
+    return m / (np.sqrt(v) + eps)
+
+
+def _mut_adam_eps_in_root(m, v, beta1, beta2, eps, step):
+    return (m / (1 - beta1 ** step)) / np.sqrt(v / (1 - beta2 ** step) + eps)
+
+
+def _mut_adam_decay_new_p(p, g, m, v, *, lr, beta1, beta2, eps, weight_decay, step):
+    m1, v1 = ao.adamw_moments(m, v, g, beta1, beta2)
+    return (p - lr * ao.adamw_direction(m1, v1, beta1, beta2, eps, step)) * (1 - lr * weight_decay), m1, v1
+
+
+def _mut_adam_decay_without_lr(p, g, m, v, *, lr, beta1, beta2, eps, weight_decay, step):
+    m1, v1 = ao.adamw_moments(m, v, g, beta1, beta2)
+    return p * (1 - weight_decay) - lr * ao.adamw_direction(m1, v1, beta1, beta2, eps, step), m1, v1
+
+
+ADAMW_MUTANTS = [
+    ("adamw_moments", _mut_adam_swapped_betas),
+    ("adamw_moments", _mut_adam_abs_second_moment),
+    ("adamw_direction", _mut_adam_no_bias_correction),
+    ("adamw_direction", _mut_adam_eps_in_root),
+    ("adamw_step", _mut_adam_decay_new_p),
+    ("adamw_step", _mut_adam_decay_without_lr),
+]
+
+
+def test_unmutated_adamw_oracle_passes_its_pins():
+    assert not _adamw_pins_fail()
+
+
+@pytest.mark.parametrize("name,mutant", ADAMW_MUTANTS, ids=[f"{n}-{m.__name__}" for n, m in ADAMW_MUTANTS])
+def test_planted_adamw_mistake_is_caught(monkeypatch, name, mutant):
+    monkeypatch.setattr(ao, name, mutant)
+    assert _adamw_pins_fail(), f"mutant {mutant.__name__} of {name} slipped through the pins"
