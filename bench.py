@@ -385,11 +385,12 @@ def run_ours(args, world, rank, local):
 
     ws = api.Workspace(dev)
     stream = torch.cuda.current_stream(dev)
-    kw = dict(lr=w.lr, beta=w.beta, weight_decay=w.weight_decay, nesterov=w.nesterov, coeffs=coeffs,
-              workspace=ws, stream=stream)
+    # the descriptors are built once (PreparedMuonStep); every step is one C ABI call
+    step_fn = api.PreparedMuonStep(ps, gs, ms, lr=w.lr, beta=w.beta, weight_decay=w.weight_decay,
+                                   nesterov=w.nesterov, coeffs=coeffs, workspace=ws)
 
     for _ in range(args.warmup):
-        api.muon_step(ps, gs, ms, **kw)
+        step_fn(stream)
     torch.cuda.synchronize()
 
     L = _lib.lib()
@@ -404,7 +405,7 @@ def run_ours(args, world, rank, local):
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        api.muon_step(ps, gs, ms, **kw)
+        step_fn(stream)
     e1.record(stream)
     torch.cuda.synchronize()
     clocks.mark(False)
@@ -413,12 +414,27 @@ def run_ours(args, world, rank, local):
     clk = clocks.stop()
     ms_step = dist_max(ms_step, world)
 
+    # ---- step-time spread: events between steps only (launches inside a step keep their
+    # programmatic overlap); p10 / p50 / p90 over up to 200 steps
+    spread_steps = max(1, min(args.steps, 200))
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(spread_steps + 1)]
+    torch.cuda.synchronize()
+    evs[0].record(stream)
+    for i in range(spread_steps):
+        step_fn(stream)
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize()
+    per_step = sorted(evs[i].elapsed_time(evs[i + 1]) for i in range(spread_steps))
+    pct = lambda f: per_step[min(len(per_step) - 1, int(f * len(per_step)))]  # noqa: E731
+    spread = {"p10": round(pct(0.10), 4), "p50": round(pct(0.50), 4), "p90": round(pct(0.90), 4),
+              "steps": spread_steps}
+
     # ---- per-kernel breakdown: a second pass with an event pair around every launch
     prof_steps = max(1, min(args.steps, 50))
     torch.cuda.synchronize()
     _lib.check(L.muon_profile_begin(), "muon_profile_begin")
     for _ in range(prof_steps):
-        api.muon_step(ps, gs, ms, **kw)
+        step_fn(stream)
     torch.cuda.synchronize()
     kms = (ctypes.c_double * 6)()
     kcount = (ctypes.c_int64 * 6)()
@@ -433,7 +449,7 @@ def run_ours(args, world, rank, local):
         pin_p = torch.empty_like(P, device="cpu").pin_memory()
         for _ in range(2):
             G.copy_(pin_g, non_blocking=True)
-            api.muon_step(ps, gs, ms, **kw)
+            step_fn(stream)
             pin_p.copy_(P, non_blocking=True)
         torch.cuda.synchronize()
         barrier(world)
@@ -443,7 +459,7 @@ def run_ours(args, world, rank, local):
         f0.record(stream)
         for _ in range(e2e_steps):
             G.copy_(pin_g, non_blocking=True)
-            api.muon_step(ps, gs, ms, **kw)
+            step_fn(stream)
             pin_p.copy_(P, non_blocking=True)
         f1.record(stream)
         torch.cuda.synchronize()
@@ -515,11 +531,164 @@ def run_ours(args, world, rank, local):
             "d2h_bytes_per_step": P.numel() * P.element_size()},
         "gpu_launches": int(launches_per_step * args.steps),
         "profiled_steps": prof_steps,
+        "ms_per_step_spread": spread,
     }
     if world == 1 and not args.no_cpu_baseline:
         cms, sample = oracle_sample_ms(w)
         line["cpu_baseline"] = {"value": round(cms, 1), "unit": "ms", "cores": blas_threads(), "kind": "oracle",
                                 "sample": sample}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ AdamW path
+
+ADAMW_HYPER = dict(lr=1e-3, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1)
+ADAMW_BYTES_PER_ELEM = 24  # bf16 p read + written, fp32 g read, fp32 m and v read + written
+
+
+def adamw_layout():
+    """(name, numel, offset) of each tensor in flat buffers; offsets are multiples of 8
+    elements, so every view keeps 16-byte alignment (the vector path)."""
+    out, off = [], 0
+    for name, n in inputs.gpt2_124m_adamw_tensors():
+        out.append((name, n, off))
+        off += (n + 7) // 8 * 8
+    return out, off
+
+
+def adamw_oracle_sample_ms(step=2):
+    """The fp64 oracle's AdamW step on a bounded sample (the first 2^21 elements of the token
+    embedding), scaled to the whole parameter set by element count."""
+    import numpy as np
+
+    from oracle import adamw_oracle as ao
+
+    layout, _ = adamw_layout()
+    total = sum(n for _, n, _ in layout)
+    k = 1 << 21
+    rng = np.random.default_rng(0)
+    p = 0.02 * rng.standard_normal(k)
+    g = 1e-3 * rng.standard_normal(k)
+    m = 0.1 * g
+    v = 0.05 * g * g
+    t0 = time.perf_counter()
+    ao.adamw_step(p, g, m, v, step=step, **{"lr": ADAMW_HYPER["lr"], "beta1": ADAMW_HYPER["beta1"],
+                                           "beta2": ADAMW_HYPER["beta2"], "eps": ADAMW_HYPER["eps"],
+                                           "weight_decay": ADAMW_HYPER["weight_decay"]})
+    dt = time.perf_counter() - t0
+    sample = (f"the fp64 oracle's AdamW step on the first {k} elements of the token embedding, "
+              f"scaled to all {total} elements")
+    return dt * 1e3 * total / k, sample
+
+
+def run_adamw(args, world, rank, local):
+    import torch
+
+    from newton_schulz_11_b200 import api, build
+
+    build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    layout, flat = adamw_layout()
+    P = torch.empty(flat, dtype=torch.bfloat16, device=dev)
+    G = torch.zeros(flat, dtype=torch.float32, device=dev)
+    M = torch.zeros(flat, dtype=torch.float32, device=dev)
+    V = torch.zeros(flat, dtype=torch.float32, device=dev)
+    ps = [P[o:o + n] for _, n, o in layout]
+    gs = [G[o:o + n] for _, n, o in layout]
+    ms = [M[o:o + n] for _, n, o in layout]
+    vs = [V[o:o + n] for _, n, o in layout]
+    with torch.no_grad():
+        for i, (_, n, o) in enumerate(layout):
+            ps[i].copy_(inputs.adamw_param_torch(i, n, dev))
+            gs[i].copy_(inputs.adamw_grad_torch(1, i, n, dev))
+    numel = sum(n for _, n, _ in layout)
+    stream = torch.cuda.current_stream(dev)
+    adamw = api.PreparedAdamW(ps, gs, ms, vs, lr=ADAMW_HYPER["lr"], betas=(ADAMW_HYPER["beta1"], ADAMW_HYPER["beta2"]),
+                              eps=ADAMW_HYPER["eps"], weight_decay=ADAMW_HYPER["weight_decay"])
+    t = 0
+    for _ in range(args.warmup):
+        t += 1
+        adamw(t, stream)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(gpu_id_for(local))
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.mark(True)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        t += 1
+        adamw(t, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark(False)
+    barrier(world)
+    ms_step = dist_max(e0.elapsed_time(e1) / args.steps, world)
+    clk = clocks.stop()
+    e2e = None
+    if not args.no_e2e:
+        pin_g = G.cpu().pin_memory()
+        pin_p = torch.empty_like(P, device="cpu").pin_memory()
+        e2e_steps = max(1, min(args.steps, 50))
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        f0.record(stream)
+        for _ in range(e2e_steps):
+            t += 1
+            G.copy_(pin_g, non_blocking=True)
+            adamw(t, stream)
+            pin_p.copy_(P, non_blocking=True)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        e2e = {"value": round(dist_max(f0.elapsed_time(f1) / e2e_steps, world), 4), "unit": "ms",
+               "h2d_bytes_per_step": G.numel() * 4, "d2h_bytes_per_step": P.numel() * 2}
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    launches = (len(layout) + 127) // 128
+    by = ADAMW_BYTES_PER_ELEM * numel / launches
+    gbs = by / (ms_step / launches * 1e-3) / 1e9
+    line = {
+        "metric": "adamw_step_ms", "value": round(ms_step, 4), "unit": "ms", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": inputs.ADAMW_WORKLOAD, "tensors": len(layout), "params": numel, "param_dtype": "bf16",
+                   "l2": "inputs larger than L2 (%.2f GB moved per step)" % (ADAMW_BYTES_PER_ELEM * numel / 1e9),
+                   "parallelism": "replicas" if world > 1 else "single"},
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None, "kernel": "muon_adamw_kernel",
+                     "peak_source": peak_src + " copy", "algorithmic_bytes_per_launch": int(by)},
+        "clocks": clk, "e2e": e2e, "gpu_launches": launches * args.steps,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        cms, sample = adamw_oracle_sample_ms()
+        line["cpu_baseline"] = {"value": round(cms, 1), "unit": "ms", "cores": blas_threads(), "kind": "oracle",
+                                "sample": sample}
+    print(json.dumps(line), flush=True)
+
+
+def run_adamw_reference(args, world, rank):
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        adamw_oracle_sample_ms()
+    runs = [adamw_oracle_sample_ms() for _ in range(args.steps)]
+    value = statistics.median(r[0] for r in runs)
+    layout, _ = adamw_layout()
+    line = {
+        "impl": "reference", "metric": "adamw_step_ms", "value": round(value, 3), "unit": "ms", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(value, 3), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": inputs.ADAMW_WORKLOAD, "tensors": len(layout), "params": sum(n for _, n, _ in layout)},
+        "cpu_baseline": {"value": round(value, 3), "unit": "ms", "cores": blas_threads(), "kind": "oracle",
+                         "sample": runs[0][1]},
+        "e2e": {"value": round(value, 3), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
     print(json.dumps(line), flush=True)
 
 
@@ -533,6 +702,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer pass (for workloads whose inputs do not fit pinned host memory)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", default="muon", choices=["muon", "adamw"],
+                    help="muon: the Muon step (default); adamw: the AdamW step of the non-matrix parameters")
     ap.add_argument("--matrices", type=int, default=0,
                     help="run only the first K matrices of the workload (a small case of the same kernels)")
     args = ap.parse_args()
@@ -541,11 +712,11 @@ def main():
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
-        run_reference(args, world, rank)
+        (run_adamw_reference if args.path == "adamw" else run_reference)(args, world, rank)
         return
     world, rank, local = dist_setup(args)
     try:
-        run_ours(args, world, rank, local)
+        (run_adamw if args.path == "adamw" else run_ours)(args, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -186,6 +186,37 @@ muon_status_t muon_profile_begin(void);
 muon_status_t muon_profile_end(double* ms_by_kind, int64_t* launches_by_kind, int kinds);
 
 /*
+ * AdamW for the parameters Muon does not take: biases, norm gains and embeddings.
+ * "14 - modded-nanogpt: the Speedrun Community", section 3: the canonical Muon setup is
+ * hybrid, Muon on the 2-D matmul weights and AdamW on the rest.  The pages give no
+ * formula; this is the textbook decoupled-decay AdamW with bias correction:
+ *   m <- beta1 m + (1 - beta1) g,  v <- beta2 v + (1 - beta2) g^2
+ *   p <- p (1 - lr wd) - (lr / (1 - beta1^step)) m / (sqrt(v / (1 - beta2^step)) + eps)
+ * Each tensor is contiguous and flattened to `numel` elements.
+ *   param       in/out, fp32 or bf16 (param_dtype), aligned to its element size
+ *   grad        in, fp32
+ *   exp_avg     in/out fp32 (m), exp_avg_sq in/out fp32 (v); start from zeros
+ * All device pointers; 16-byte aligned buffers take the vector path.  Buffers written
+ * (param, exp_avg, exp_avg_sq) may overlap no other buffer of the call.
+ * Hyperparameters: finite, lr >= 0, 0 <= beta1, beta2 < 1, eps > 0, weight_decay >= 0,
+ * step >= 1 (the 1-based count of updates including this one).  Asynchronous on `stream`;
+ * on a validation error nothing is queued.
+ */
+typedef struct {
+  void*        param;
+  const float* grad;
+  float*       exp_avg;
+  float*       exp_avg_sq;
+  int64_t      numel;
+  int32_t      param_dtype;   /* MUON_F32 or MUON_BF16 */
+  int32_t      reserved;      /* set to 0 */
+} muon_adamw_tensor_t;
+
+muon_status_t muon_adamw_step(const muon_adamw_tensor_t* tensors, int n, float lr, float beta1,
+                              float beta2, float eps, float weight_decay, int64_t step,
+                              void* stream);
+
+/*
  * Newton-Schulz without a caller-supplied workspace, for callers that cannot allocate
  * device memory: code that runs inside another framework's memory pool or allocator
  * (where a cudaMalloc of its own would fragment that pool, or is forbidden), plugins

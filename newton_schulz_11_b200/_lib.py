@@ -37,6 +37,7 @@ EXPORTS = (
     "muon_profile_begin",
     "muon_profile_end",
     "muon_newton_schulz_static",
+    "muon_adamw_step",
 )
 
 KIND_NAMES = ("momentum", "norm", "gram", "poly", "apply", "apply_last")
@@ -55,6 +56,18 @@ class MuonMatrix(ctypes.Structure):
         ("ld_mom", ctypes.c_int64),
         ("param_dtype", ctypes.c_int32),
         ("shape_scale", ctypes.c_float),
+    ]
+
+
+class MuonAdamwTensor(ctypes.Structure):
+    _fields_ = [
+        ("param", ctypes.c_void_p),
+        ("grad", ctypes.c_void_p),
+        ("exp_avg", ctypes.c_void_p),
+        ("exp_avg_sq", ctypes.c_void_p),
+        ("numel", ctypes.c_int64),
+        ("param_dtype", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
     ]
 
 
@@ -130,6 +143,10 @@ def lib() -> ctypes.CDLL:
         h.muon_profile_begin.argtypes = []
         h.muon_profile_end.restype = ctypes.c_int
         h.muon_profile_end.argtypes = [P(ctypes.c_double), P(ctypes.c_int64), ctypes.c_int]
+        h.muon_adamw_step.restype = ctypes.c_int
+        h.muon_adamw_step.argtypes = [P(MuonAdamwTensor), ctypes.c_int, ctypes.c_float, ctypes.c_float,
+                                      ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_int64,
+                                      ctypes.c_void_p]
         h.muon_newton_schulz_static.restype = ctypes.c_int
         h.muon_newton_schulz_static.argtypes = [P(MuonMatrix), ctypes.c_int, ctypes.c_int, P(ctypes.c_float),
                                                 ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p]

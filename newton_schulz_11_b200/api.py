@@ -11,7 +11,7 @@ from typing import List, Optional, Sequence, Tuple
 import torch
 
 from . import _lib
-from ._lib import MuonError, MuonLibraryError, MuonMatrix, MuonScratchView, check, lib  # noqa: F401
+from ._lib import MUON_BF16, MUON_F32, MuonAdamwTensor, MuonError, MuonLibraryError, MuonMatrix, MuonScratchView, check, lib  # noqa: F401,E501
 
 # "NanoGPT Speedrun" README, zeroth_power_via_newtonschulz5 listing: (a, b, c), 5 steps, eps.
 QUINTIC = (3.4445, -4.7750, 2.0315)
@@ -208,6 +208,104 @@ def newton_schulz_static(Gs: Sequence[torch.Tensor], *, coeffs=None, eps: float 
     check(lib().muon_newton_schulz_static(arr, len(Gs), steps, table, float(eps), st_ptr, s),
           "muon_newton_schulz_static")
     return outs
+
+
+def _adamw_descriptors(params, grads, exp_avgs, exp_avg_sqs):
+    params, grads, exp_avgs, exp_avg_sqs = list(params), list(grads), list(exp_avgs), list(exp_avg_sqs)
+    n = len(params)
+    if n == 0 or not (len(grads) == len(exp_avgs) == len(exp_avg_sqs) == n):
+        raise ValueError("params, grads, exp_avgs and exp_avg_sqs must be non-empty lists of equal length")
+    device = params[0].device
+    arr = (MuonAdamwTensor * n)()
+    for i, (p, g, m, v) in enumerate(zip(params, grads, exp_avgs, exp_avg_sqs)):
+        for t, what in ((p, "param"), (g, "grad"), (m, "exp_avg"), (v, "exp_avg_sq")):
+            if t.device != device or t.device.type != "cuda":
+                raise ValueError(f"{what} {i} is not on {device}")
+            if not t.is_contiguous():
+                raise ValueError(f"{what} {i} must be contiguous")
+            if t.numel() != p.numel():
+                raise ValueError(f"{what} {i} has {t.numel()} elements, param has {p.numel()}")
+        if p.dtype not in (torch.float32, torch.bfloat16):
+            raise ValueError(f"param {i} must be float32 or bfloat16")
+        for t, what in ((g, "grad"), (m, "exp_avg"), (v, "exp_avg_sq")):
+            if t.dtype != torch.float32:
+                raise ValueError(f"{what} {i} must be float32")
+        arr[i].param = p.data_ptr()
+        arr[i].grad = g.data_ptr()
+        arr[i].exp_avg = m.data_ptr()
+        arr[i].exp_avg_sq = v.data_ptr()
+        arr[i].numel = p.numel()
+        arr[i].param_dtype = MUON_BF16 if p.dtype == torch.bfloat16 else MUON_F32
+    return arr, n, device
+
+
+def adamw_step(params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor], exp_avgs: Sequence[torch.Tensor],
+               exp_avg_sqs: Sequence[torch.Tensor], *, lr: float, step: int, betas=(0.9, 0.999),
+               eps: float = 1e-8, weight_decay: float = 0.0, stream=None) -> None:
+    """AdamW on a grouped list of contiguous tensors (the parameters Muon does not take).
+
+    params fp32 or bf16; grads, exp_avgs, exp_avg_sqs fp32 of the same numel; `step` is the
+    1-based count of updates including this one.  One launch per 128 tensors.  For a fixed
+    set of tensors stepped repeatedly, PreparedAdamW avoids rebuilding the descriptors.
+    """
+    arr, n, device = _adamw_descriptors(params, grads, exp_avgs, exp_avg_sqs)
+    b1, b2 = betas
+    check(lib().muon_adamw_step(arr, n, float(lr), float(b1), float(b2), float(eps), float(weight_decay),
+                                int(step), _stream_handle(device, stream)), "muon_adamw_step")
+
+
+class PreparedMuonStep:
+    """muon_step for a fixed set of tensors: the descriptor array, coefficient table and
+    workspace are built once, so each call is one C ABI call (no per-call Python checks).
+    The tensors must keep their storage (same data pointers) between calls."""
+
+    def __init__(self, params, grads, moms, *, lr: float, beta: float = 0.95, weight_decay: float = 0.0,
+                 nesterov: bool = True, coeffs=None, eps: float = DEFAULT_EPS, shape_scales=None, outs=None,
+                 workspace: Optional[Workspace] = None):
+        if not (len(params) == len(grads) == len(moms)) or len(grads) == 0:
+            raise ValueError("params, grads and moms must be equally long, non-empty lists")
+        self._keep = (list(params), list(grads), list(moms), None if outs is None else list(outs))
+        self._arr = _descriptors(params, grads, moms, outs, shape_scales, ns_only=False)
+        self._n = len(grads)
+        self._table, self._steps = _coeff_array(coeffs if coeffs is not None else quintic_table())
+        self.device = grads[0].device
+        need = ctypes.c_size_t(0)
+        check(lib().muon_workspace_size(self._arr, self._n, ctypes.byref(need)), "muon_workspace_size")
+        self._ws = workspace or default_workspace(self.device)
+        self._ptr, size = self._ws.ensure(int(need.value), _stream_handle(self.device, None))
+        self._bytes = min(size, int(need.value))
+        self._hyper = (float(lr), float(beta), float(weight_decay), 1 if nesterov else 0)
+        self._eps = float(eps)
+        self._fn = lib().muon_step
+
+    def __call__(self, stream=None) -> None:
+        lr, beta, wd, nest = self._hyper
+        st = self._fn(self._arr, self._n, lr, beta, wd, nest, self._steps, self._table, self._eps, self._ptr,
+                      self._bytes, _stream_handle(self.device, stream))
+        if st != 0:
+            check(st, "muon_step")
+
+    @property
+    def workspace(self) -> Workspace:
+        return self._ws
+
+
+class PreparedAdamW:
+    """adamw_step for a fixed set of contiguous tensors: the descriptor array is built and
+    checked once; each call passes the 1-based step count to one C ABI call."""
+
+    def __init__(self, params, grads, exp_avgs, exp_avg_sqs, *, lr: float, betas=(0.9, 0.999),
+                 eps: float = 1e-8, weight_decay: float = 0.0):
+        self._keep = (list(params), list(grads), list(exp_avgs), list(exp_avg_sqs))
+        self._arr, self._n, self.device = _adamw_descriptors(*self._keep)
+        self._hyper = (float(lr), float(betas[0]), float(betas[1]), float(eps), float(weight_decay))
+        self._fn = lib().muon_adamw_step
+
+    def __call__(self, step: int, stream=None) -> None:
+        lr, b1, b2, eps, wd = self._hyper
+        st = self._fn(self._arr, self._n, lr, b1, b2, eps, wd, int(step), _stream_handle(self.device, stream))
+        if st != 0:
+            check(st, "muon_adamw_step")
 
 
 def scratch_view(shapes: Sequence[Tuple[int, int]], index: int, workspace_bytes: int) -> MuonScratchView:

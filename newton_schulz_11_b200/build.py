@@ -21,7 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmuon_b200.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 
-SOURCES = ["muon_elementwise.cu", "muon_ns_gemm.cu", "muon_host.cu"]
+SOURCES = ["muon_elementwise.cu", "muon_ns_gemm.cu", "muon_host.cu", "muon_adamw.cu"]
 HEADERS = ["muon_device.cuh", "muon_params.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

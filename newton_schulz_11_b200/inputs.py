@@ -196,6 +196,47 @@ def weight_torch(workload: Workload, mat: int, device):
     return w.to(torch.bfloat16) if workload.param_dtype == "bf16" else w
 
 
+# ------------------------------------------------------------------ AdamW tensors
+
+def gpt2_124m_adamw_tensors() -> List[Tuple[str, int]]:
+    """The parameters of the GPT-2 124M layout that the hybrid setup gives to AdamW (the
+    1-D ones and the embeddings): token embedding 50257 x 768, position embedding
+    1024 x 768, and per layer the two LayerNorm gains and biases and the four linear
+    biases, plus the final LayerNorm.  Returned as (name, numel)."""
+    d, vocab, ctx, layers = 768, 50257, 1024, 12
+    out = [("wte", vocab * d), ("wpe", ctx * d)]
+    for i in range(layers):
+        out += [(f"h{i}.ln_1.weight", d), (f"h{i}.ln_1.bias", d), (f"h{i}.attn.c_attn.bias", 3 * d),
+                (f"h{i}.attn.c_proj.bias", d), (f"h{i}.ln_2.weight", d), (f"h{i}.ln_2.bias", d),
+                (f"h{i}.mlp.c_fc.bias", 4 * d), (f"h{i}.mlp.c_proj.bias", d)]
+    out += [("ln_f.weight", d), ("ln_f.bias", d)]
+    return out
+
+
+ADAMW_WORKLOAD = "gpt2-124m-adamw-params"
+ADAMW_INDEX = 10  # seed component, distinct from the Muon workloads
+
+
+def adamw_grad_torch(step: int, i: int, numel: int, device, std: float = 1e-3):
+    """fp32 gradient of AdamW tensor i at `step`: std * N(0, 1), seeded like the Muon inputs."""
+    import torch
+
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(np.random.SeedSequence([ROOT_SEED, ADAMW_INDEX, step, i, ROLE_GRAD_NOISE])
+                        .generate_state(1, np.uint64)[0] >> 1))
+    return torch.randn(numel, generator=gen, device=device, dtype=torch.float32).mul_(std)
+
+
+def adamw_param_torch(i: int, numel: int, device):
+    """bf16 parameter of AdamW tensor i: 0.02 * N(0, 1)."""
+    import torch
+
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(np.random.SeedSequence([ROOT_SEED, ADAMW_INDEX, 0, i, ROLE_W])
+                        .generate_state(1, np.uint64)[0] >> 1))
+    return torch.randn(numel, generator=gen, device=device, dtype=torch.float32).mul_(0.02).to(torch.bfloat16)
+
+
 def scaled_workload(workload: Workload, shapes: Sequence[Tuple[int, int]], name: Optional[str] = None) -> Workload:
     """Same value recipe and hyperparameters on other shapes (small parity cases)."""
     return dataclasses.replace(workload, shapes=tuple(shapes), name=name or workload.name + "-scaled")

@@ -135,3 +135,32 @@ def test_device_status_stays_ok():
     ws = api.Workspace(gs[0].device)
     api.muon_step(Ws, gs, ms, lr=0.02, workspace=ws)
     assert api.device_status(ws) == (_lib.MUON_OK, 0)
+
+
+def test_prepared_calls_match_one_shot_calls():
+    """PreparedMuonStep / PreparedAdamW reuse their descriptors; results are bit-identical
+    to the one-shot calls, over consecutive steps."""
+    require_gpu()
+    from newton_schulz_11_b200 import api
+
+    Ws, gs, ms = _set(SHAPES)
+    W1, m1 = _clone(Ws), _clone(ms)
+    W2, m2 = _clone(Ws), _clone(ms)
+    prep = api.PreparedMuonStep(W2, gs, m2, lr=0.02, weight_decay=0.01)
+    for _ in range(2):
+        api.muon_step(W1, gs, m1, lr=0.02, weight_decay=0.01)
+        prep()
+    for a, b in zip(W1 + m1, W2 + m2):
+        assert torch.equal(a, b)
+
+    g = [torch.randn(n, device="cuda") for n in (5, 4096, 70001)]
+    p1 = [torch.randn(x.numel(), device="cuda").to(torch.bfloat16) for x in g]
+    p2 = _clone(p1)
+    st1 = [[torch.zeros_like(x) for x in g] for _ in range(2)]
+    st2 = [[torch.zeros_like(x) for x in g] for _ in range(2)]
+    prep_a = api.PreparedAdamW(p2, g, st2[0], st2[1], lr=1e-3, betas=(0.9, 0.95), weight_decay=0.1)
+    for t in (1, 2, 3):
+        api.adamw_step(p1, g, st1[0], st1[1], lr=1e-3, step=t, betas=(0.9, 0.95), weight_decay=0.1)
+        prep_a(t)
+    for a, b in zip(p1 + st1[0] + st1[1], p2 + st2[0] + st2[1]):
+        assert torch.equal(a, b)
