@@ -37,7 +37,11 @@ KINDS = ("momentum", "norm", "gram", "poly", "apply", "apply_last")
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture of
 # the benchmarked workload, keyed by kernel kind; valid only while the kernel sources hash to
 # `source_hash` (see profiles/).  Filled in from the committed ncu summary.
-NCU_TRAFFIC = {"source_hash": None, "workload": DEFAULT_WORKLOAD, "bytes_per_launch": {}}
+NCU_TRAFFIC = {"source_hash": "cb211889b266f68e", "workload": DEFAULT_WORKLOAD,
+               "bytes_per_launch": {"momentum": 1302197504, "norm": 29952, "gram": 210061000,
+                                    "poly": 126210000, "apply": 712098000, "apply_last": 744524288}}
+# the same for the AdamW path (workload gpt2-124m-adamw-params, one launch per step)
+NCU_TRAFFIC_ADAMW = {"source_hash": "cb211889b266f68e", "bytes_per_launch": 893366784}
 
 
 def kernel_source_hash() -> str:
@@ -661,7 +665,10 @@ def run_adamw(args, world, rank, local):
                    "l2": "inputs larger than L2 (%.2f GB moved per step)" % (ADAMW_BYTES_PER_ELEM * numel / 1e9),
                    "parallelism": "replicas" if world > 1 else "single"},
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None, "kernel": "muon_adamw_kernel",
+                     "frac": round(gbs / peaks["hbm_gbs"], 4),
+                     "traffic": NCU_TRAFFIC_ADAMW["bytes_per_launch"]
+                     if NCU_TRAFFIC_ADAMW["source_hash"] == kernel_source_hash() else None,
+                     "kernel": "muon_adamw_kernel",
                      "peak_source": peak_src + " copy", "algorithmic_bytes_per_launch": int(by)},
         "clocks": clk, "e2e": e2e, "gpu_launches": launches * args.steps,
     }

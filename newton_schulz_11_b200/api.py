@@ -308,6 +308,20 @@ class PreparedAdamW:
             check(st, "muon_adamw_step")
 
 
+def head_blocks(W: torch.Tensor, head_dim: int, heads_per_block: int = 2, dim: int = 0) -> List[torch.Tensor]:
+    """Views of W split into blocks of `heads_per_block` heads along `dim` (0: the rows of a
+    Q/K/V projection, 1: the columns of the output projection).  Each block is a strided
+    2-D view of W's storage (no copy), so a grouped muon_step over the blocks orthogonalises
+    every block as its own matrix and updates W in place -- per-head (heads_per_block=1)
+    or paired-head (2) Muon."""
+    if W.dim() != 2:
+        raise ValueError("W must be 2-D")
+    size = head_dim * heads_per_block
+    if W.shape[dim] % size:
+        raise ValueError(f"dimension {dim} of W ({W.shape[dim]}) is not a multiple of {size}")
+    return list(torch.split(W, size, dim=dim))
+
+
 def scratch_view(shapes: Sequence[Tuple[int, int]], index: int, workspace_bytes: int) -> MuonScratchView:
     n = len(shapes)
     arr = (MuonMatrix * n)()

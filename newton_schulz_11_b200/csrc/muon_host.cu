@@ -146,8 +146,11 @@ void prof_stop(int i, cudaStream_t s) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// A strided 2-D region of memory: `rows` rows of `width` bytes, `pitch` bytes apart.
 struct Range {
-  uintptr_t lo, hi;
+  uintptr_t lo, hi;  // first byte, one past the last byte
+  uintptr_t pitch, width;
+  int64_t rows;
   bool written;
 };
 
@@ -155,7 +158,25 @@ void add_range(std::vector<Range>& v, const void* base, int64_t rows, int64_t co
                bool written) {
   const uintptr_t lo = reinterpret_cast<uintptr_t>(base);
   const uintptr_t hi = lo + static_cast<uintptr_t>(((rows - 1) * ld + cols) * static_cast<int64_t>(elt));
-  v.push_back({lo, hi, written});
+  v.push_back({lo, hi, static_cast<uintptr_t>(ld) * elt, static_cast<uintptr_t>(cols) * elt, rows, written});
+}
+
+// Whether two regions whose byte spans overlap share a byte.  Regions with the same pitch
+// (sub-blocks of one matrix, e.g. per-head column blocks) are tested exactly: row by row
+// in the frame of the one that starts first.  Other pairs count as sharing.
+bool regions_share_bytes(const Range& a, const Range& b) {
+  const Range& x = a.lo <= b.lo ? a : b;
+  const Range& y = a.lo <= b.lo ? b : a;
+  if (x.pitch != y.pitch || x.width > x.pitch || y.width > y.pitch) return true;
+  const uintptr_t d = y.lo - x.lo;
+  const int64_t q = static_cast<int64_t>(d / x.pitch);  // y's first row, in x's rows
+  const uintptr_t off = d % x.pitch;                     // y's column offset in bytes
+  auto rows_meet = [&](int64_t first) { return first < x.rows && first + y.rows > 0; };
+  // the part of each y row that lies in parent row q + k
+  if (off < x.width && rows_meet(q)) return true;
+  // the part that spills into parent row q + k + 1 (starting at column 0)
+  if (off + y.width > x.pitch && rows_meet(q + 1)) return true;
+  return false;
 }
 
 muon_status_t validate(const muon_matrix_t* mats, int n, bool ns_only) {
@@ -185,15 +206,13 @@ muon_status_t validate(const muon_matrix_t* mats, int n, bool ns_only) {
     add_range(ranges, t.param, t.rows, t.cols, t.ld_param, pe, true);
     add_range(ranges, t.momentum, t.rows, t.cols, t.ld_mom, 4, true);
   }
-  // No written buffer may overlap any other buffer.
+  // No written buffer may share a byte with any other buffer.  Pairs whose byte spans
+  // overlap are tested exactly (blocks of one matrix interleave without sharing bytes).
   std::sort(ranges.begin(), ranges.end(), [](const Range& a, const Range& b) { return a.lo < b.lo; });
-  uintptr_t max_any = 0, max_written = 0;
-  for (const Range& r : ranges) {
-    if (r.lo < max_written) return MUON_ERR_INVALID_ARG;
-    if (r.written && r.lo < max_any) return MUON_ERR_INVALID_ARG;
-    max_any = std::max(max_any, r.hi);
-    if (r.written) max_written = std::max(max_written, r.hi);
-  }
+  for (size_t i = 0; i < ranges.size(); ++i)
+    for (size_t j = i + 1; j < ranges.size() && ranges[j].lo < ranges[i].hi; ++j)
+      if ((ranges[i].written || ranges[j].written) && regions_share_bytes(ranges[i], ranges[j]))
+        return MUON_ERR_INVALID_ARG;
   return MUON_OK;
 }
 

@@ -23,3 +23,15 @@ def load_golden(name):
 @pytest.fixture
 def golden():
     return load_golden
+
+
+def cuda_present() -> bool:
+    """True when a CUDA device is visible.  Host-side tests that hand fake device pointers to
+    an entry point make the calls that would pass validation only when this is False: with
+    a device present such a call would launch kernels on addresses that do not exist."""
+    try:
+        import torch
+
+        return torch.cuda.is_available()
+    except Exception:  # pragma: no cover
+        return False

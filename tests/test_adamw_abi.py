@@ -5,6 +5,7 @@ import ctypes
 import pytest
 
 from newton_schulz_11_b200 import _lib
+from tests.conftest import cuda_present
 
 
 @pytest.fixture(scope="module")
@@ -29,8 +30,10 @@ def call(L, arr, n=None, lr=1e-3, b1=0.9, b2=0.999, eps=1e-8, wd=0.0, step=1):
 
 
 def test_valid_call_reaches_the_device_check(L):
+    if cuda_present():
+        pytest.skip("fake device pointers: only where no kernel can run")
     st = call(L, tensors([10, 1000, 3]))
-    assert st in (_lib.MUON_ERR_NO_DEVICE, _lib.MUON_ERR_CUDA, _lib.MUON_OK)
+    assert st in (_lib.MUON_ERR_NO_DEVICE, _lib.MUON_ERR_CUDA)
 
 
 def test_rejects_bad_arguments(L):
@@ -55,7 +58,8 @@ def test_rejects_bad_arguments(L):
     bad = tensors([10, 10]); bad[1].param = bad[0].grad + 8  # a write over another tensor's grad
     assert call(L, bad) == E.MUON_ERR_INVALID_ARG
     ok = tensors([10, 10]); ok[1].grad = ok[0].grad  # two tensors reading one grad is allowed
-    assert call(L, ok) in (E.MUON_ERR_NO_DEVICE, E.MUON_ERR_CUDA, E.MUON_OK)
+    if not cuda_present():
+        assert call(L, ok) in (E.MUON_ERR_NO_DEVICE, E.MUON_ERR_CUDA)
 
 
 def test_struct_layout_matches_header():
