@@ -164,3 +164,19 @@ def test_prepared_calls_match_one_shot_calls():
         prep_a(t)
     for a, b in zip(p1 + st1[0] + st1[1], p2 + st2[0] + st2[1]):
         assert torch.equal(a, b)
+
+
+def test_sharded_muon_on_one_rank_is_the_plain_step():
+    """Without a process group (one rank) the sharded step owns every matrix and runs the
+    library's grouped step: bit-identical to muon_step."""
+    require_gpu()
+    from newton_schulz_11_b200 import api
+    from newton_schulz_11_b200.distributed import ShardedMuon
+
+    Ws, gs, ms = _set(SHAPES)
+    W1, m1 = _clone(Ws), _clone(ms)
+    W2, m2 = _clone(Ws), _clone(ms)
+    api.muon_step(W1, gs, m1, lr=0.02, weight_decay=0.01)
+    ShardedMuon(W2, gs, m2, lr=0.02, weight_decay=0.01)()
+    for a, b in zip(W1 + m1, W2 + m2):
+        assert torch.equal(a, b)
