@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define MUON_ABI_VERSION 1
+#define MUON_ABI_VERSION 2
 #define MUON_MAX_NS_STEPS 16
 
 typedef enum {
@@ -92,15 +92,23 @@ typedef struct {
   float        shape_scale;  /* multiplier on lr; <= 0 selects sqrt(max(1, rows / cols)) */
 } muon_matrix_t;
 
-/* Where one matrix's scratch lives inside the workspace (diagnostics and tests). */
+/*
+ * Where one matrix's scratch lives inside the workspace (diagnostics and tests).
+ * X is carried between iterations as hi + lo: hi = bf16(x) (the tensor-core operand) and
+ * lo = x - hi as a signed 8-bit fixed-point residual in units of 2^(e - 15), with e the
+ * exponent of hi (|x - hi| <= 2^(e - 8), so |lo| <= 127 after rounding to nearest even
+ * and clamping); x = hi + lo * 2^(e - 15), and lo = 0 where hi's biased exponent is
+ * below 16.
+ */
 typedef struct {
   uint64_t x_hi_offset[2];   /* bf16 [rows x x_ld]: ping-pong high parts of X */
-  uint64_t x_lo_offset;      /* bf16 [rows x x_ld]: low part of X */
+  uint64_t x_lo_offset;      /* int8 [rows x x_lo_ld]: low part of X, see above */
   uint64_t a_offset;         /* bf16 [m x a_ld]: A = X X^T of the latest iteration */
   uint64_t b_offset;         /* bf16 [m x a_ld]: B = b A + c A A of the latest iteration */
   uint64_t scale_offset;     /* fp32: 1 / (||u||_F + eps) */
   uint64_t norm_offset;      /* fp32: ||u||_F */
   int64_t  x_ld;             /* elements */
+  int64_t  x_lo_ld;          /* bytes (= elements) */
   int64_t  a_ld;             /* elements */
   int32_t  wave;             /* matrices are processed in waves that reuse the workspace */
   int32_t  transposed;       /* 1 when rows > cols (X is the transpose of the stored matrix) */

@@ -80,6 +80,7 @@ class MuonScratchView(ctypes.Structure):
         ("scale_offset", ctypes.c_uint64),
         ("norm_offset", ctypes.c_uint64),
         ("x_ld", ctypes.c_int64),
+        ("x_lo_ld", ctypes.c_int64),
         ("a_ld", ctypes.c_int64),
         ("wave", ctypes.c_int32),
         ("transposed", ctypes.c_int32),

@@ -387,6 +387,50 @@ __device__ __forceinline__ void split_hi_lo2(float x0, float x1, uint32_t& hi, u
   lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
+// ---- X as hi + lo with an 8-bit lo
+// hi = bf16(x); lo = x - hi as a signed fixed-point residual in units of 2^(e - 15), e the
+// exponent of hi: |x - hi| <= 2^(e - 8) gives |lo| <= 128, rounded to nearest even and
+// clamped to [-127, 127]; x = hi + lo * 2^(e - 15).  The worst-case residual error,
+// 2^(e - 16), is the same as that of a bf16 residual.  Where hi's biased exponent is below
+// 16 (|x| < 2^-111) lo is 0.
+
+// 2^(e - 15) for the bf16 hi (bit pattern in the low 16 bits), or 0 (integer exponent
+// arithmetic only).
+__device__ __forceinline__ float lo8_unit(uint32_t hi16) {
+  const int32_t eb = static_cast<int32_t>((hi16 << 16) & 0x7F800000u);
+  return __int_as_float(max(eb - (15 << 23), 0));
+}
+
+// The 8-bit residual of x against its bf16 hi (bit pattern hi16), as a byte.  The scaled
+// residual is clamped, then rounded to nearest even by adding 1.5 * 2^23, which leaves the
+// integer's two's complement in the low bits of the sum (full-rate float and integer ops).
+__device__ __forceinline__ uint32_t lo8_encode(float x, uint32_t hi16) {
+  const uint32_t hb = hi16 << 16;
+  const uint32_t eb = hb & 0x7F800000u;
+  const float r = x - __uint_as_float(hb);                                   // exact
+  const float t = fminf(fmaxf(r * __uint_as_float(0x86800000u - eb), -127.f), 127.f);  // r * 2^(15 - e)
+  const uint32_t q = __float_as_uint(t + 12582912.f) & 0xFFu;
+  return eb >= (16u << 23) ? q : 0u;
+}
+
+// x from a bf16 hi (bits hi16) and its 8-bit residual (byte lo8).
+__device__ __forceinline__ float lo8_decode(uint32_t hi16, uint32_t lo8) {
+  const uint32_t k = static_cast<uint32_t>(static_cast<int32_t>(lo8 << 24) >> 24);  // sign-extended
+  const float q = __uint_as_float(0x4B400000u + k) - 12582912.f;
+  return fmaf(q, lo8_unit(hi16), __uint_as_float(hi16 << 16));
+}
+
+// Four values at once: hi as two bf16x2 words (h01: x0 low, x1 high; h23 likewise) and the
+// four residual bytes in one word (x0 in the lowest byte).
+__device__ __forceinline__ void split_hi_lo8x4(float x0, float x1, float x2, float x3, uint32_t& h01, uint32_t& h23,
+                                               uint32_t& l4) {
+  const __nv_bfloat162 a = __floats2bfloat162_rn(x0, x1), b = __floats2bfloat162_rn(x2, x3);
+  h01 = *reinterpret_cast<const uint32_t*>(&a);
+  h23 = *reinterpret_cast<const uint32_t*>(&b);
+  l4 = lo8_encode(x0, h01 & 0xFFFFu) | (lo8_encode(x1, h01 >> 16) << 8) | (lo8_encode(x2, h23 & 0xFFFFu) << 16) |
+       (lo8_encode(x3, h23 >> 16) << 24);
+}
+
 // L2 prefetch of the line holding `p`.
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));

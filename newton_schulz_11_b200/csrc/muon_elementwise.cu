@@ -2,7 +2,8 @@
 //
 //   m' = beta m + g                        ("14 - modded-nanogpt", section 3, muon_step)
 //   u  = g + beta m'  (Nesterov) or m'     ("NanoGPT Speedrun" README, practices list)
-//   hi = bf16(u), lo = bf16(u - hi)        Newton-Schulz input, unscaled
+//   hi = bf16(u), lo = 8-bit residual      Newton-Schulz input, unscaled (lo in units of
+//                                          2^(e - 15), e the exponent of hi)
 //   partial[chunk] = sum of u^2            for ||u||_F of the listing's G.norm()
 //
 // followed by a per-matrix finalisation s = 1 / (||u||_F + eps) in a fixed order
@@ -75,14 +76,10 @@ __global__ void __launch_bounds__(kEwThreads) muon_momentum_kernel(const __grid_
       float u2 = ew_one(g.z, m.z, beta, nesterov, ns_only);
       float u3 = ew_one(g.w, m.w, beta, nesterov, ns_only);
       if (!ns_only) __stcs(reinterpret_cast<float4*>(mp), m);
-      uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
-      split_hi_lo(u0, h0, l0);
-      split_hi_lo(u1, h1, l1);
-      split_hi_lo(u2, h2, l2);
-      split_hi_lo(u3, h3, l3);
-      const int64_t o = static_cast<int64_t>(r) * t.ldx + c;
-      *reinterpret_cast<uint2*>(t.hi + o) = make_uint2(h0 | (h1 << 16), h2 | (h3 << 16));
-      *reinterpret_cast<uint2*>(t.lo + o) = make_uint2(l0 | (l1 << 16), l2 | (l3 << 16));
+      uint32_t h01, h23, l4;
+      split_hi_lo8x4(u0, u1, u2, u3, h01, h23, l4);
+      *reinterpret_cast<uint2*>(t.hi + static_cast<int64_t>(r) * t.ldx + c) = make_uint2(h01, h23);
+      *reinterpret_cast<uint32_t*>(t.lo + static_cast<int64_t>(r) * t.ldl + c) = l4;
       acc = fmaf(u0, u0, acc);
       acc = fmaf(u1, u1, acc);
       acc = fmaf(u2, u2, acc);
@@ -99,11 +96,9 @@ __global__ void __launch_bounds__(kEwThreads) muon_momentum_kernel(const __grid_
       float m = ns_only ? 0.f : *mp;
       const float u = ew_one(g, m, beta, nesterov, ns_only);
       if (!ns_only) *mp = m;
-      uint32_t h, l;
-      split_hi_lo(u, h, l);
-      const int64_t o = static_cast<int64_t>(r) * t.ldx + c;
-      t.hi[o] = __ushort_as_bfloat16(static_cast<unsigned short>(h));
-      t.lo[o] = __ushort_as_bfloat16(static_cast<unsigned short>(l));
+      const uint32_t h = float_to_bf16_bits(u);
+      t.hi[static_cast<int64_t>(r) * t.ldx + c] = __ushort_as_bfloat16(static_cast<unsigned short>(h));
+      t.lo[static_cast<int64_t>(r) * t.ldl + c] = static_cast<int8_t>(lo8_encode(u, h));
       acc = fmaf(u, u, acc);
     }
   }

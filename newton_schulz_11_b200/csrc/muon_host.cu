@@ -47,6 +47,7 @@ std::atomic<long long> g_timeout_us{2000000};
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int64_t round8(int64_t x) { return (x + 7) / 8 * 8; }
+int64_t round16(int64_t x) { return (x + 15) / 16 * 16; }
 int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
 // ---------------------------------------------------------------- device facts
@@ -106,6 +107,20 @@ bool encode_map(CUtensorMap* map, void* base, int64_t count, int64_t rows, int64
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The 8-bit lo buffer: 64 x 128 boxes (64 bytes of a row, 128 rows), 64-byte swizzle.
+bool encode_map_lo(CUtensorMap* map, void* base, int64_t count, int64_t rows, int64_t cols, int64_t ldl) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(count)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(ldl), static_cast<cuuint64_t>(ldl * rows)};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -233,6 +248,7 @@ muon_status_t validate_hyper(float lr, float beta, float wd, int nesterov, int n
 
 struct ClassPlan {
   int64_t rows = 0, cols = 0, m = 0, n = 0, ldx = 0, lda = 0;
+  int64_t ldl = 0;  // row stride of the 8-bit lo buffer (bytes, multiple of 16)
   int tall = 0;
   std::vector<int> mats;  // global indices
   size_t off_hi[2] = {0, 0}, off_lo = 0, off_a = 0, off_b = 0;
@@ -267,6 +283,7 @@ WavePlan layout_wave(const muon_matrix_t* mats, const std::vector<int>& idx) {
       c->n = std::max(t.rows, t.cols);
       c->tall = t.rows > t.cols ? 1 : 0;
       c->ldx = round8(t.cols);
+      c->ldl = round16(t.cols);
       c->lda = round8(c->m);
     }
     c->mats.push_back(i);
@@ -290,13 +307,14 @@ WavePlan layout_wave(const muon_matrix_t* mats, const std::vector<int>& idx) {
   off = align_up(off + 4 * static_cast<size_t>(w.total_chunks), kBufAlign);
   for (auto& c : w.classes) {
     const size_t xb = static_cast<size_t>(c.mats.size()) * c.rows * c.ldx * 2;
+    const size_t lb = static_cast<size_t>(c.mats.size()) * c.rows * c.ldl;
     const size_t ab = static_cast<size_t>(c.mats.size()) * c.m * c.lda * 2;
     c.off_hi[0] = off;
     off = align_up(off + xb, kBufAlign);
     c.off_hi[1] = off;
     off = align_up(off + xb, kBufAlign);
     c.off_lo = off;
-    off = align_up(off + xb, kBufAlign);
+    off = align_up(off + lb, kBufAlign);
     c.off_a = off;
     off = align_up(off + ab, kBufAlign);
     c.off_b = off;
@@ -383,7 +401,7 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
     const int count = static_cast<int>(c.mats.size());
     __nv_bfloat16* hi0 = reinterpret_cast<__nv_bfloat16*>(ws + c.off_hi[0]);
     __nv_bfloat16* hi1 = reinterpret_cast<__nv_bfloat16*>(ws + c.off_hi[1]);
-    __nv_bfloat16* lo = reinterpret_cast<__nv_bfloat16*>(ws + c.off_lo);
+    int8_t* lo = reinterpret_cast<int8_t*>(ws + c.off_lo);
     __nv_bfloat16* ab = reinterpret_cast<__nv_bfloat16*>(ws + c.off_a);
     __nv_bfloat16* bb = reinterpret_cast<__nv_bfloat16*>(ws + c.off_b);
     if (!encode_map(&op_hi[ci][0], hi0, count, c.rows, c.cols, c.ldx, 128) ||
@@ -392,7 +410,7 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
         !encode_map(&op_b[ci], bb, count, c.m, c.m, c.lda, 128) ||
         !encode_map(&st_hi[ci][0], hi0, count, c.rows, c.cols, c.ldx, 64) ||
         !encode_map(&st_hi[ci][1], hi1, count, c.rows, c.cols, c.ldx, 64) ||
-        !encode_map(&st_lo[ci], lo, count, c.rows, c.cols, c.ldx, 64) ||
+        !encode_map_lo(&st_lo[ci], lo, count, c.rows, c.cols, c.ldl) ||
         !encode_map(&st_a[ci], ab, count, c.m, c.m, c.lda, 64) ||
         !encode_map(&st_b[ci], bb, count, c.m, c.m, c.lda, 64))
       return MUON_ERR_CUDA;
@@ -408,6 +426,8 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
     d.lda = static_cast<int32_t>(c.lda);
     d.mat_base = local;
     d.x_stride = c.rows * c.ldx;
+    d.lo_stride = c.rows * c.ldl;
+    d.ldl = static_cast<int32_t>(c.ldl);
     d.a_stride = c.m * c.lda;
     d.x_lo = lo;
     d.a_buf = ab;
@@ -438,12 +458,13 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
       e.g = t.grad;
       e.m = t.momentum;
       e.hi = hi0 + static_cast<int64_t>(k) * d.x_stride;
-      e.lo = lo + static_cast<int64_t>(k) * d.x_stride;
+      e.lo = lo + static_cast<int64_t>(k) * d.lo_stride;
       e.ld_g = t.ld_grad;
       e.ld_m = t.ld_mom;
       e.rows = d.rows;
       e.cols = d.cols;
       e.ldx = d.ldx;
+      e.ldl = d.ldl;
       e.rows_per_chunk = w.rows_per_chunk[local];
       e.chunk_begin = w.chunk_begin[local];
       e.nchunks = w.nchunks[local];
@@ -753,12 +774,13 @@ muon_status_t muon_scratch_view(const muon_matrix_t* mats, int n, int index, siz
         const size_t aoff = k * static_cast<size_t>(c.m * c.lda) * 2;
         view->x_hi_offset[0] = c.off_hi[0] + xoff;
         view->x_hi_offset[1] = c.off_hi[1] + xoff;
-        view->x_lo_offset = c.off_lo + xoff;
+        view->x_lo_offset = c.off_lo + k * static_cast<size_t>(c.rows * c.ldl);
         view->a_offset = c.off_a + aoff;
         view->b_offset = c.off_b + aoff;
         view->scale_offset = w.off_scale + 4 * static_cast<size_t>(local);
         view->norm_offset = w.off_norm + 4 * static_cast<size_t>(local);
         view->x_ld = c.ldx;
+        view->x_lo_ld = c.ldl;
         view->a_ld = c.lda;
         view->wave = static_cast<int32_t>(wi);
         view->transposed = c.tall;

@@ -56,14 +56,15 @@ namespace muon {
 //     Gram        five stages; two 32 KB output staging buffers (stores of one quarter
 //                 drain while the next is written)
 //     polynomial  three stages; two output buffers; the tile's A block (64 KB) staged
-//     apply       three stages; the tile's hi and lo (128 KB) staged and updated in place
+//     apply       four stages; the tile's hi (64 KB) and 8-bit lo (32 KB) staged and
+//                 updated in place
 template <int MODE, bool SMALL = false>
 struct Lay {
   static constexpr bool kSym = MODE == kGram || MODE == kPoly;
   static constexpr int TM = 256;  // pair tile rows (128 per CTA)
   static constexpr int TN = 256;  // pair tile columns = UMMA N
   static constexpr int BK = SMALL ? 64 : 128;
-  static constexpr int S = (SMALL && MODE == kGram) ? 5 : 3;
+  static constexpr int S = !SMALL ? 3 : (MODE == kGram ? 5 : (kSym ? 3 : 4));
   static constexpr int NEPI = 8;
   static constexpr int kBox64 = 64 * 64 * 2;       // one 64 x 64 box: 8 KB
   static constexpr int kHalf = kBM * kBox * 2;      // one 64 x 128 box: 16 KB
@@ -73,7 +74,7 @@ struct Lay {
   static constexpr int kRing = S * kStageBytes;
   // streamed: one 64-column quarter of this CTA's 128 x 256 tile at a time (symmetric
   // modes D_q and T_q, apply hi_q and lo_q); staged: see above
-  static constexpr int kEpi = !SMALL ? 2 * kHalf : (MODE == kGram ? 4 * kHalf : 8 * kHalf);
+  static constexpr int kEpi = !SMALL ? 2 * kHalf : (MODE == kGram ? 4 * kHalf : (kSym ? 8 * kHalf : 6 * kHalf));
   static constexpr int kBarOff = kRing + kEpi;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;
   static constexpr int kEpiThreads = 32 * NEPI;
@@ -254,6 +255,47 @@ __device__ __forceinline__ void load_row32(const __nv_bfloat16* row, int valid, 
   }
 }
 
+// 32 consecutive bytes of a row of the 8-bit lo buffer (two 16-byte loads), zero past
+// `valid` columns or when `live` is false.  `row` is 16-byte aligned.
+__device__ __forceinline__ void load_row32_u8(const int8_t* row, int valid, bool live, uint4 (&w)[2]) {
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    if (live && 16 * q < valid)
+      w[q] = __ldg(reinterpret_cast<const uint4*>(row) + q);
+    else
+      w[q] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  if (live && valid < 32 && valid > 0) {
+    uint32_t* e = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int k = valid - 4 * j;  // bytes of word j that lie inside the row
+      if (k <= 0) e[j] = 0u;
+      else if (k < 4) e[j] &= (1u << (8 * k)) - 1u;
+    }
+  }
+}
+
+constexpr int kLoBlock = kBM * 64;  // one quarter of 8-bit lo: 128 rows x 64 bytes
+
+// A staged 128-row x 64-byte block of the 8-bit lo buffer (one TMA box, 64-byte swizzle):
+// row r at r * 64 B, its 16-byte chunk c (0..3) at chunk c ^ ((r >> 1) & 3).
+__device__ __forceinline__ uint32_t lo8_chunk(int r, int c) {
+  return static_cast<uint32_t>(r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
+}
+
+// Decodes 32 values of a row: x_j = hi_j + lo_j 2^(e_j - 15) for the bf16 pairs in `h`
+// (16 words, element 2i in the low half of word i) and the residual bytes in `l`
+// (8 words, element j in byte j % 4 of word j / 4).
+__device__ __forceinline__ void decode32(const uint32_t* h, const uint32_t* l, float (&x)[32]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t lw = l[i >> 1] >> (16 * (i & 1));
+    x[2 * i] = lo8_decode(h[i] & 0xFFFFu, lw & 0xFFu);
+    x[2 * i + 1] = lo8_decode(h[i] >> 16, (lw >> 8) & 0xFFu);
+  }
+}
+
 // Stores 128 x 64 staged at Q (two boxes) at rows row0.., columns col0..
 __device__ __forceinline__ void store_q(const CUtensorMap* map, const uint8_t* q, int row0, int col0, int mat) {
   tma_store_3d(map, q, col0, row0, mat);
@@ -390,27 +432,25 @@ __device__ __forceinline__ bool load_w_segment(const FinalParams& p, const Class
 }
 
 // X update for the 32 tile columns [c0, c0 + 32) of this CTA's tile row r, with the old
-// hi/lo pair already in registers: x = s (a (hi + lo) + acc).  kApply returns the new
-// pair packed (hb, lb); kApplyLast updates W and/or writes O in global memory.
+// hi (16 bf16x2 words) and lo (8 words of residual bytes) already in registers:
+// x = s (a (hi + lo) + acc).  kApply returns the new pair packed (hb: 16 bf16x2 words,
+// lb: 8 words of bytes); kApplyLast updates W and/or writes O in global memory.
 template <int MODE>
 __device__ __forceinline__ void apply_quarter(const typename ParamsOf<MODE>::type& p, const ClassDesc& cd,
                                               const Tile& tl, int rank, int r, int c0, uint32_t tcol,
-                                              const uint4 (&xh4)[4], const uint4 (&xl4)[4], float s,
-                                              uint32_t (&hb)[16], uint32_t (&lb)[16]) {
+                                              const uint4 (&xh4)[4], const uint4 (&xl4)[2], float s,
+                                              uint32_t (&hb)[16], uint32_t (&lb)[8]) {
   uint32_t v[32];
   tmem_ld_32x32b_x32(tcol, v);
-  tmem_wait_ld();
-  const uint32_t* xh = reinterpret_cast<const uint32_t*>(xh4);
-  const uint32_t* xl = reinterpret_cast<const uint32_t*>(xl4);
   float x[32];
+  decode32(reinterpret_cast<const uint32_t*>(xh4), reinterpret_cast<const uint32_t*>(xl4), x);
+  tmem_wait_ld();
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    x[2 * i] = s * fmaf(p.a, lo_bf16(xh[i]) + lo_bf16(xl[i]), __uint_as_float(v[2 * i]));
-    x[2 * i + 1] = s * fmaf(p.a, hi_bf16(xh[i]) + hi_bf16(xl[i]), __uint_as_float(v[2 * i + 1]));
-  }
+  for (int j = 0; j < 32; ++j) x[j] = s * fmaf(p.a, x[j], __uint_as_float(v[j]));
   if constexpr (MODE == kApply) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) split_hi_lo2(x[2 * i], x[2 * i + 1], hb[i], lb[i]);
+    for (int k = 0; k < 8; ++k)
+      split_hi_lo8x4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3], hb[2 * k], hb[2 * k + 1], lb[k]);
   } else {
     (void)hb;
     (void)lb;
@@ -418,7 +458,8 @@ __device__ __forceinline__ void apply_quarter(const typename ParamsOf<MODE>::typ
   }
 }
 
-// Staged variant of the same update: the old pair is read from the staged region; kApply
+// Staged variant of the same update: the old pair is read from the staged region (hi at
+// hib in the 128-byte swizzle, lo at lob in 64-byte-swizzled 8 KB quarter blocks); kApply
 // writes the new pair back in place (the region is then stored by TMA), kApplyLast updates
 // W and/or writes O (w_pre: this thread's W segment, loaded ahead, or nullptr).
 template <int MODE>
@@ -427,36 +468,36 @@ __device__ __forceinline__ void apply_staged(const typename ParamsOf<MODE>::type
                                              uint8_t* lob, float s, const uint4* w_pre = nullptr) {
   uint32_t v[32];
   tmem_ld_32x32b_x32(tcol, v);
-  uint4 xh4[4], xl4[4];
+  uint4 xh4[4], xl4[2];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint32_t o = region_chunk(r, (c0 >> 3) + q);
-    xh4[q] = *reinterpret_cast<const uint4*>(hib + o);
-    xl4[q] = *reinterpret_cast<const uint4*>(lob + o);
-  }
-  tmem_wait_ld();
-  const uint32_t* xh = reinterpret_cast<const uint32_t*>(xh4);
-  const uint32_t* xl = reinterpret_cast<const uint32_t*>(xl4);
+  for (int q = 0; q < 4; ++q) xh4[q] = *reinterpret_cast<const uint4*>(hib + region_chunk(r, (c0 >> 3) + q));
+  // quarter c0 / 64 of the lo block; this thread's 32 bytes are chunks 2 h, 2 h + 1 of its row
+  uint8_t* lq = lob + ((c0 >> 6) << 13);
+  const int lc = (c0 & 63) >> 4;
+#pragma unroll
+  for (int q = 0; q < 2; ++q) xl4[q] = *reinterpret_cast<const uint4*>(lq + lo8_chunk(r, lc + q));
   float x[32];
+  decode32(reinterpret_cast<const uint32_t*>(xh4), reinterpret_cast<const uint32_t*>(xl4), x);
+  tmem_wait_ld();
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    x[2 * i] = fmaf(p.a, lo_bf16(xh[i]) + lo_bf16(xl[i]), __uint_as_float(v[2 * i]));
-    x[2 * i + 1] = fmaf(p.a, hi_bf16(xh[i]) + hi_bf16(xl[i]), __uint_as_float(v[2 * i + 1]));
-  }
+  for (int j = 0; j < 32; ++j) x[j] = fmaf(p.a, x[j], __uint_as_float(v[j]));
   if (s != 1.f) {  // iteration 0 only (uniform)
 #pragma unroll
     for (int j = 0; j < 32; ++j) x[j] *= s;
   }
   if constexpr (MODE == kApply) {
-    uint32_t hb[16], lb[16];
+    uint32_t hb[16], lb[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) split_hi_lo2(x[2 * i], x[2 * i + 1], hb[i], lb[i]);
+    for (int k = 0; k < 8; ++k)
+      split_hi_lo8x4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3], hb[2 * k], hb[2 * k + 1], lb[k]);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint32_t o = region_chunk(r, (c0 >> 3) + q);
-      *reinterpret_cast<uint4*>(hib + o) = make_uint4(hb[4 * q], hb[4 * q + 1], hb[4 * q + 2], hb[4 * q + 3]);
-      *reinterpret_cast<uint4*>(lob + o) = make_uint4(lb[4 * q], lb[4 * q + 1], lb[4 * q + 2], lb[4 * q + 3]);
-    }
+    for (int q = 0; q < 4; ++q)
+      *reinterpret_cast<uint4*>(hib + region_chunk(r, (c0 >> 3) + q)) =
+          make_uint4(hb[4 * q], hb[4 * q + 1], hb[4 * q + 2], hb[4 * q + 3]);
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+      *reinterpret_cast<uint4*>(lq + lo8_chunk(r, lc + q)) = make_uint4(lb[4 * q], lb[4 * q + 1], lb[4 * q + 2],
+                                                                        lb[4 * q + 3]);
   } else {
     write_update<MODE>(p, cd, tl, rank, r, c0, x, w_pre);
   }
@@ -666,15 +707,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
     const bool leader = threadIdx.x == 64;  // also the thread that waits on the barriers
     const uint32_t tempty0 = map_to_rank(smem_u32(tempty), 0);
     uint8_t* hib = epi;
-    uint8_t* lob = epi + 4 * L::kHalf;
+    uint8_t* lob = epi + 4 * L::kHalf;  // four 8 KB blocks of 8-bit lo, one per quarter
     int acc = 0;
     uint32_t aph = 0;
     uint32_t pending = 0, pend_par = 0;  // leader: quarter loads not yet waited for, and their parity
     auto load_quarter = [&](const Tile& nx, int q, uint32_t par) {
       const int row0 = L::TM * nx.I + kBM * rank, col0 = L::TN * nx.J;
-      mbar_arrive_expect_tx(&efull[q], 2 * L::kHalf);
+      mbar_arrive_expect_tx(&efull[q], L::kHalf + kLoBlock);
       load_region_quarter(hib, &p.map_in[nx.cls], &efull[q], q, row0, col0, nx.mat);
-      load_region_quarter(lob, &p.map_out2[nx.cls], &efull[q], q, row0, col0, nx.mat);
+      tma_load_3d(lob + q * kLoBlock, &p.map_out2[nx.cls], &efull[q], col0 + 64 * q, row0, nx.mat);
       pending |= 1u << q;
       pend_par = (pend_par & ~(1u << q)) | (par << q);
     };
@@ -759,7 +800,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
           named_barrier(1, NT);  // quarter q is final
           if (leader) {
             store_region(&p.map_out[tl.cls], hib, q, 1, row0, col0, tl.mat);
-            store_region(&p.map_out2[tl.cls], lob, q, 1, row0, col0, tl.mat);
+            tma_store_3d(&p.map_out2[tl.cls], lob + q * kLoBlock, col0 + 64 * q, row0, tl.mat);
             bulk_commit();
             // the stores of quarter q - 1 have read their boxes: refill them
             if (q > 0) {
@@ -907,10 +948,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
       // Epilogue inputs come straight from global memory (L2) into registers; they are
       // requested before the accumulator is waited for.
       uint4 in_a[4][4];  // polynomial: A, the four quarters' 32 columns of this row
-      uint4 ch[4], cl[4];  // apply: hi and lo of the first quarter
+      uint4 ch[4], cl[2];  // apply: hi and 8-bit lo of the first quarter
       const int rb = 2 * tl.I + rank;
       const int Rx = L::TM * tl.I + kBM * rank + r;
       const int64_t xoff = tl.mat * cd.x_stride + static_cast<int64_t>(Rx) * cd.ldx;
+      const int64_t loff = tl.mat * cd.lo_stride + static_cast<int64_t>(Rx) * cd.ldl;
       const int Cb = L::TN * tl.J + 32 * h;
       if constexpr (MODE == kPoly) {
         const int Ra = kBM * rb + r;
@@ -923,7 +965,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
         }
       } else if constexpr (!kSym) {
         load_row32(cd.x_hi_cur + xoff + Cb, cd.cols - Cb, Rx < cd.rows, ch);
-        load_row32(cd.x_lo + xoff + Cb, cd.cols - Cb, Rx < cd.rows, cl);
+        load_row32_u8(cd.x_lo + loff + Cb, cd.cols - Cb, Rx < cd.rows, cl);
       }
       // The next tile's epilogue inputs start moving from HBM into L2 now, so that its
       // loads above hit L2 (apply: hi and lo; polynomial: A).
@@ -940,8 +982,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             tma_prefetch_l2_3d(mh, L::TN * nx.J + 64 * c, rn, nx.mat);
-            tma_prefetch_l2_3d(&p.map_out2[nx.cls], L::TN * nx.J + 64 * c, rn, nx.mat);
-            tma_prefetch_l2_3d(&p.map_out2[nx.cls], L::TN * nx.J + 64 * c, rn + 64, nx.mat);
+            tma_prefetch_l2_3d(&p.map_out2[nx.cls], L::TN * nx.J + 64 * c, rn, nx.mat);  // 128 rows of lo
           }
         }
       }
@@ -986,13 +1027,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
         const int row0 = L::TM * tl.I + kBM * rank;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          uint4 nh[4], nl[4];
+          uint4 nh[4], nl[2];
           if (q < 3) {
             const int Cn = Cb + 64 * (q + 1);
             load_row32(cd.x_hi_cur + xoff + Cn, cd.cols - Cn, Rx < cd.rows, nh);
-            load_row32(cd.x_lo + xoff + Cn, cd.cols - Cn, Rx < cd.rows, nl);
+            load_row32_u8(cd.x_lo + loff + Cn, cd.cols - Cn, Rx < cd.rows, nl);
           }
-          uint32_t hb[16], lb[16];
+          uint32_t hb[16], lb[8];
           apply_quarter<MODE>(p, cd, tl, rank, r, 64 * q + 32 * h, tacc + 64 * q + 32 * h, ch, cl, sc, hb, lb);
           if (q == 3) {
             tc_fence_before();
@@ -1006,22 +1047,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
             for (int k = 0; k < 4; ++k) {
               const uint32_t o = q_chunk(r, 4 * h + k);
               *reinterpret_cast<uint4*>(Q + o) = make_uint4(hb[4 * k], hb[4 * k + 1], hb[4 * k + 2], hb[4 * k + 3]);
-              *reinterpret_cast<uint4*>(Tst + o) = make_uint4(lb[4 * k], lb[4 * k + 1], lb[4 * k + 2], lb[4 * k + 3]);
             }
+            // the quarter's 8-bit lo: one 128-row x 64-byte block at Tst, chunks 2 h, 2 h + 1
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+              *reinterpret_cast<uint4*>(Tst + lo8_chunk(r, 2 * h + k)) =
+                  make_uint4(lb[4 * k], lb[4 * k + 1], lb[4 * k + 2], lb[4 * k + 3]);
             fence_proxy_async_smem();
             named_barrier(1, NT);
             if (leader) {
               store_q(&p.map_out[tl.cls], Q, row0, L::TN * tl.J + 64 * q, tl.mat);
-              store_q(&p.map_out2[tl.cls], Tst, row0, L::TN * tl.J + 64 * q, tl.mat);
+              tma_store_3d(&p.map_out2[tl.cls], Tst, L::TN * tl.J + 64 * q, row0, tl.mat);
               bulk_commit();
             }
           }
           if (q < 3) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              ch[k] = nh[k];
-              cl[k] = nl[k];
-            }
+            for (int k = 0; k < 4; ++k) ch[k] = nh[k];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) cl[k] = nl[k];
           }
         }
       }

@@ -51,11 +51,14 @@ struct ClassDesc {
   int32_t out_rows, out_cols;
   int32_t a_mn, b_mn;     // operand majorness: 0 = K-major, 1 = MN-major
   int32_t i_fast;         // tile order: row tiles vary fastest
-  int64_t x_stride;       // elements between consecutive matrices in the X buffers
+  int64_t x_stride;       // elements between consecutive matrices in the hi buffers
+  int64_t lo_stride;      // bytes between consecutive matrices in the lo buffer
   int64_t a_stride;       // elements between consecutive matrices in A / B
+  int32_t ldl;            // row stride of the lo buffer (bytes, multiple of 16)
+  int32_t pad_;
   __nv_bfloat16* x_hi_cur;   // hi part read this iteration
   __nv_bfloat16* x_hi_next;  // hi part written this iteration
-  __nv_bfloat16* x_lo;       // lo part, updated in place
+  int8_t* x_lo;              // lo part (8-bit residual of hi), updated in place
   __nv_bfloat16* a_buf;
   __nv_bfloat16* b_buf;
 };
@@ -75,7 +78,7 @@ struct GemmParams {
   CUtensorMap map_a[kMaxClasses];     // operand A of the launch, per class (64 x 128 boxes)
   CUtensorMap map_b[kMaxClasses];     // operand B (64 x 128 boxes)
   CUtensorMap map_out[kMaxClasses];   // epilogue store: Gram -> A, polynomial -> B, apply -> next hi
-  CUtensorMap map_out2[kMaxClasses];  // epilogue store: apply -> lo (64 x 64 boxes, like map_out)
+  CUtensorMap map_out2[kMaxClasses];  // apply: lo (8-bit, 64 x 128 boxes, 64-byte swizzle), load and store
   CUtensorMap map_in[kMaxClasses];    // staged apply: the current hi as epilogue input (64 x 64)
   ClassDesc cls[kMaxClasses];
   int32_t num_classes;
@@ -98,9 +101,9 @@ struct EwMat {
   const float* g;
   float* m;
   __nv_bfloat16* hi;
-  __nv_bfloat16* lo;
+  int8_t* lo;               // 8-bit residual of hi, row stride ldl bytes
   int64_t ld_g, ld_m;
-  int32_t rows, cols, ldx;
+  int32_t rows, cols, ldx, ldl;
   int32_t rows_per_chunk;
   int32_t chunk_begin;
   int32_t nchunks;

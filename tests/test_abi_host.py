@@ -38,7 +38,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.muon_abi_version() == 1
+    assert L.muon_abi_version() == 2
     for code in range(9):
         assert L.muon_status_str(code).decode() not in ("", "unknown status")
     assert L.muon_status_str(99).decode() == "unknown status"
@@ -78,10 +78,11 @@ def step(L, arr, n=None, lr=0.02, beta=0.95, wd=0.0, nesterov=1, steps=5, c=None
 def test_workspace_size_matches_layout(L):
     st, b = ws_size(L, mats_of([(768, 3072)]))
     assert st == 0
-    x = 768 * 3072 * 2
+    x = 768 * 3072 * 2  # each bf16 hi buffer
+    lo = 768 * 3072      # the 8-bit lo buffer
     a = 768 * 768 * 2
-    assert b >= 3 * x + 2 * a
-    assert b < 3 * x + 2 * a + 64 * 1024
+    assert b >= 2 * x + lo + 2 * a
+    assert b < 2 * x + lo + 2 * a + 64 * 1024
 
 
 def test_workspace_size_for_every_workload(L):
@@ -109,11 +110,12 @@ def test_scratch_view_tall_and_padding(L):
     st, full = ws_size(L, arr)
     v = MuonScratchView()
     assert L.muon_scratch_view(arr, 3, 2, full, ctypes.byref(v)) == 0
-    assert v.transposed == 1 and v.x_ld == 40 and v.a_ld == 40
-    assert v.x_hi_offset[0] % 16 == 0 and v.a_offset % 16 == 0
+    assert v.transposed == 1 and v.x_ld == 40 and v.a_ld == 40 and v.x_lo_ld == 48
+    assert v.x_hi_offset[0] % 16 == 0 and v.a_offset % 16 == 0 and v.x_lo_offset % 16 == 0
     v0 = MuonScratchView()
     L.muon_scratch_view(arr, 3, 0, full, ctypes.byref(v0))
     assert v.x_hi_offset[0] - v0.x_hi_offset[0] == 100 * 40 * 2  # same class, next slot
+    assert v.x_lo_offset - v0.x_lo_offset == 100 * 48
 
 
 def test_validation_rejects_bad_descriptors_without_cuda(L):

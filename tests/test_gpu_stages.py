@@ -8,7 +8,7 @@ at one kernel (elementwise, Gram, polynomial or apply) and one orientation.
 import numpy as np
 import pytest
 
-from tests.gpu_util import require_gpu, rel_fro, to_np, torch, ws_matrix, ws_scalar
+from tests.gpu_util import lo8_unit, require_gpu, rel_fro, to_np, torch, ws_lo8, ws_matrix, ws_scalar
 
 pytestmark = pytest.mark.gpu
 
@@ -35,7 +35,8 @@ def run_ns(G, coeffs):
 def scratch(ws, view, rows, cols, which_hi):
     m = min(rows, cols)
     hi = ws_matrix(ws.buf, view.x_hi_offset[which_hi], rows, cols, view.x_ld)
-    lo = ws_matrix(ws.buf, view.x_lo_offset, rows, cols, view.x_ld)
+    lo, _ = ws_lo8(ws.buf, view.x_lo_offset, rows, cols, view.x_lo_ld, hi)
+    lo = lo.float()
     A = ws_matrix(ws.buf, view.a_offset, m, m, view.a_ld)
     B = ws_matrix(ws.buf, view.b_offset, m, m, view.a_ld)
     s = ws_scalar(ws.buf, view.scale_offset)
@@ -70,9 +71,20 @@ def test_one_iteration_stage_by_stage(shape):
     assert view.transposed == int(tall)
     hi, lo, A, B, s, nrm = scratch(ws, view, rows, cols, 0)
 
-    # elementwise: hi + lo reproduces G, norm and scale
+    # elementwise: hi = bf16(G) and lo = the 8-bit residual, exactly as the format states
     Gd = G.double()
-    assert ((hi + lo).double() - Gd).abs().max().item() <= 2 ** -15 * Gd.abs().max().item()
+    assert torch.equal(hi, G.to(torch.bfloat16).float())
+    _, q = ws_lo8(ws.buf, view.x_lo_offset, rows, cols, view.x_lo_ld, hi)
+    unit = lo8_unit(hi)
+    q_ref = torch.where(unit > 0, torch.round((Gd - hi.double()) / torch.where(unit > 0, unit, 1.0)),
+                        torch.zeros_like(unit)).clamp(-127, 127)
+    bad = q != q_ref
+    if bad.any():
+        i, j = [int(v) for v in bad.nonzero()[0]]
+        raise AssertionError(f"8-bit lo differs from round-half-even((x - hi) / 2^(e - 15)) at {int(bad.sum())} "
+                             f"elements, first ({i}, {j}): got {float(q[i, j])} want {float(q_ref[i, j])}, "
+                             f"x {float(Gd[i, j])!r} hi {float(hi[i, j])!r} unit {float(unit[i, j])!r}")
+    assert ((hi.double() + q * unit) - Gd).abs().max().item() <= 2 ** -15 * Gd.abs().max().item()
     assert abs(nrm - Gd.norm().item()) <= 1e-6 * Gd.norm().item()
     assert abs(s - 1.0 / (Gd.norm().item() + 1e-7)) <= 1e-6 * s
 
