@@ -73,14 +73,14 @@ def matrix_work(rows, cols):
 
 def kind_bytes(w, kind, with_out=False):
     """Algorithmic HBM bytes of one launch of `kind` over the whole workload: every input
-    the launch needs read once, every output written once (X is a bf16 hi/lo pair)."""
+    the launch needs read once, every output written once (X is a bf16 hi and an 8-bit lo)."""
     pb = 2 if w.param_dtype == "bf16" else 4
     tot = 0
     for rows, cols in w.shapes:
         mn = rows * cols
         m = min(rows, cols)
         if kind == "momentum":
-            tot += 16 * mn           # read g, m; write m; write hi, lo
+            tot += 15 * mn           # read g, m; write m; write hi (2 B), lo (1 B)
         elif kind == "norm":
             tot += 0
         elif kind == "gram":
@@ -88,9 +88,9 @@ def kind_bytes(w, kind, with_out=False):
         elif kind == "poly":
             tot += 4 * m * m             # read A; write B
         elif kind == "apply":
-            tot += 8 * mn + 2 * m * m    # read hi, lo and B; write hi, lo
+            tot += 6 * mn + 2 * m * m    # read hi, lo and B; write hi, lo
         elif kind == "apply_last":
-            tot += (4 + 2 * pb + (4 if with_out else 0)) * mn + 2 * m * m   # read hi, lo, B; W in/out; O
+            tot += (3 + 2 * pb + (4 if with_out else 0)) * mn + 2 * m * m   # read hi, lo, B; W in/out; O
     return tot
 
 
