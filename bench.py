@@ -445,26 +445,60 @@ def run_ours(args, world, rank, local):
     _lib.check(L.muon_profile_end(kms, kcount, 6), "muon_profile_end")
     launches_per_step = sum(kcount) // prof_steps
 
-    # ---- end to end through host buffers: H2D grads, step, D2H params, every step
+    # ---- end to end through host buffers: every step copies its grads in from pinned host
+    # memory and its params out to pinned host memory.  Pipelined over two copy streams:
+    # step t + 1's grads come in (into the other of two grad buffers) and step t's params
+    # go out (from a device snapshot taken right after the step) while step t + 1 runs.
     e2e_ms = None
     if not args.no_e2e:
+        G2 = torch.empty_like(G)
+        step_fn2 = api.PreparedMuonStep(ps, [view(G2, i) for i in range(len(sizes))], ms, lr=w.lr, beta=w.beta,
+                                        weight_decay=w.weight_decay, nesterov=w.nesterov, coeffs=coeffs,
+                                        workspace=ws)
+        gbuf, steps_fn = (G, G2), (step_fn, step_fn2)
+        snap = (torch.empty_like(P), torch.empty_like(P))
         pin_g = torch.empty_like(G, device="cpu").pin_memory()
         pin_g.copy_(G.cpu())
-        pin_p = torch.empty_like(P, device="cpu").pin_memory()
-        for _ in range(2):
-            G.copy_(pin_g, non_blocking=True)
-            step_fn(stream)
-            pin_p.copy_(P, non_blocking=True)
+        pin_p = (torch.empty_like(P, device="cpu").pin_memory(), torch.empty_like(P, device="cpu").pin_memory())
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+
+        def run_e2e(n):
+            in_done, step_done, out_done = [None, None], [None, None], [None, None]
+            for t in range(n):
+                b = t % 2
+                if step_done[b] is not None:
+                    s_in.wait_event(step_done[b])      # the step that read this grad buffer is done
+                with torch.cuda.stream(s_in):
+                    gbuf[b].copy_(pin_g, non_blocking=True)
+                in_done[b] = ev()
+                in_done[b].record(s_in)
+                stream.wait_event(in_done[b])
+                steps_fn[b](stream)
+                if out_done[b] is not None:
+                    stream.wait_event(out_done[b])     # the snapshot's previous copy-out is done
+                snap[b].copy_(P, non_blocking=True)
+                step_done[b] = ev()
+                step_done[b].record(stream)
+                s_out.wait_event(step_done[b])
+                with torch.cuda.stream(s_out):
+                    pin_p[b].copy_(snap[b], non_blocking=True)
+                out_done[b] = ev()
+                out_done[b].record(s_out)
+            for e in out_done:
+                if e is not None:
+                    stream.wait_event(e)
+
+        run_e2e(2)
         torch.cuda.synchronize()
         barrier(world)
         f0 = torch.cuda.Event(enable_timing=True)
         f1 = torch.cuda.Event(enable_timing=True)
-        e2e_steps = max(1, min(args.steps, 50))
+        e2e_steps = max(2, min(args.steps, 50))
         f0.record(stream)
-        for _ in range(e2e_steps):
-            G.copy_(pin_g, non_blocking=True)
-            step_fn(stream)
-            pin_p.copy_(P, non_blocking=True)
+        s_in.wait_event(f0)
+        s_out.wait_event(f0)
+        run_e2e(e2e_steps)
         f1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = dist_max(f0.elapsed_time(f1) / e2e_steps, world)

@@ -65,6 +65,7 @@ struct Lay {
   static constexpr int TN = 256;  // pair tile columns = UMMA N
   static constexpr int BK = SMALL ? 64 : 128;
   static constexpr int S = !SMALL ? 3 : (MODE == kGram ? 5 : (kSym ? 3 : 4));
+  // epilogue warps (16 for the staged apply measured no faster than 8)
   static constexpr int NEPI = 8;
   static constexpr int kBox64 = 64 * 64 * 2;       // one 64 x 64 box: 8 KB
   static constexpr int kHalf = kBM * kBox * 2;      // one 64 x 128 box: 16 KB
@@ -284,12 +285,13 @@ __device__ __forceinline__ uint32_t lo8_chunk(int r, int c) {
   return static_cast<uint32_t>(r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
 }
 
-// Decodes 32 values of a row: x_j = hi_j + lo_j 2^(e_j - 15) for the bf16 pairs in `h`
-// (16 words, element 2i in the low half of word i) and the residual bytes in `l`
-// (8 words, element j in byte j % 4 of word j / 4).
-__device__ __forceinline__ void decode32(const uint32_t* h, const uint32_t* l, float (&x)[32]) {
+// Decodes NC values of a row: x_j = hi_j + lo_j 2^(e_j - 15) for the bf16 pairs in `h`
+// (NC / 2 words, element 2i in the low half of word i) and the residual bytes in `l`
+// (NC / 4 words, element j in byte j % 4 of word j / 4).
+template <int NC>
+__device__ __forceinline__ void decode_row(const uint32_t* h, const uint32_t* l, float (&x)[NC]) {
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
+  for (int i = 0; i < NC / 2; ++i) {
     const uint32_t lw = l[i >> 1] >> (16 * (i & 1));
     x[2 * i] = lo8_decode(h[i] & 0xFFFFu, lw & 0xFFu);
     x[2 * i + 1] = lo8_decode(h[i] >> 16, (lw >> 8) & 0xFFu);
@@ -350,26 +352,27 @@ __device__ __forceinline__ void sym_quarter(const GemmParams& p, float mul, bool
   }
 }
 
-// Final epilogue for 32 columns of one row: x holds the orthogonalised update for tile
-// columns [c0, c0 + 32) of this CTA's tile row r;  O <- x  and/or  W <- W decay - lr_scale x.
-template <int MODE>
+// Final epilogue for NC (16 or 32) columns of one row: x holds the orthogonalised update
+// for tile columns [c0, c0 + NC) of this CTA's tile row r;  O <- x  and/or
+// W <- W decay - lr_scale x.  w_pre: the bf16 W segment, loaded ahead, or nullptr.
+template <int MODE, int NC = 32>
 __device__ __forceinline__ void write_update(const FinalParams& p, const ClassDesc& cd, const Tile& tl, int rank,
-                                             int r, int c0, const float (&x)[32], const uint4* w_pre = nullptr) {
+                                             int r, int c0, const float (&x)[NC], const uint4* w_pre = nullptr) {
   const int R = Lay<MODE>::TM * tl.I + kBM * rank + r;
   const int C0 = Lay<MODE>::TN * tl.J + c0;
   const int cols = cd.cols;
   if (R >= cd.rows || C0 >= cols) return;
-  const bool full = C0 + 32 <= cols;
+  const bool full = C0 + NC <= cols;
   const UpdMat& u = p.upd[cd.mat_base + tl.mat];
   if (u.out != nullptr) {
     float* o = u.out + static_cast<int64_t>(R) * cols + C0;
     if (full && u.vec_out) {
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
+      for (int q = 0; q < NC / 4; ++q)
         reinterpret_cast<float4*>(o)[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
     } else {
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
+      for (int j = 0; j < NC; ++j)
         if (C0 + j < cols) o[j] = x[j];
     }
   }
@@ -378,27 +381,27 @@ __device__ __forceinline__ void write_update(const FinalParams& p, const ClassDe
     if (u.param_bf16) {
       __nv_bfloat16* w = static_cast<__nv_bfloat16*>(u.param) + static_cast<int64_t>(R) * u.ld_param + C0;
       if (full && u.vec_param) {
-        uint4 raw[4];
+        uint4 raw[NC / 8];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) raw[q] = w_pre != nullptr ? w_pre[q] : reinterpret_cast<const uint4*>(w)[q];
+        for (int q = 0; q < NC / 8; ++q) raw[q] = w_pre != nullptr ? w_pre[q] : reinterpret_cast<const uint4*>(w)[q];
         const uint32_t* rw = reinterpret_cast<const uint32_t*>(raw);
-        uint32_t wb[16];
+        uint32_t wb[NC / 2];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
+        for (int i = 0; i < NC / 2; ++i)
           wb[i] = pack_bf16x2(fmaf(-ls, x[2 * i], lo_bf16(rw[i]) * decay), fmaf(-ls, x[2 * i + 1], hi_bf16(rw[i]) * decay));
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
+        for (int q = 0; q < NC / 8; ++q)
           reinterpret_cast<uint4*>(w)[q] = make_uint4(wb[4 * q], wb[4 * q + 1], wb[4 * q + 2], wb[4 * q + 3]);
       } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
+        for (int j = 0; j < NC; ++j)
           if (C0 + j < cols) put_bf16(w + j, float_to_bf16_bits(fmaf(-ls, x[j], bf16_at(w + j) * decay)));
       }
     } else {
       float* w = static_cast<float*>(u.param) + static_cast<int64_t>(R) * u.ld_param + C0;
       if (full && u.vec_param) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
+        for (int q = 0; q < NC / 4; ++q) {
           float4 t = reinterpret_cast<float4*>(w)[q];
           t.x = fmaf(-ls, x[4 * q], t.x * decay);
           t.y = fmaf(-ls, x[4 * q + 1], t.y * decay);
@@ -408,26 +411,26 @@ __device__ __forceinline__ void write_update(const FinalParams& p, const ClassDe
         }
       } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
+        for (int j = 0; j < NC; ++j)
           if (C0 + j < cols) w[j] = fmaf(-ls, x[j], w[j] * decay);
       }
     }
   }
 }
 
-// The bf16 W row segment write_update reads for tile columns [c0, c0 + 32) of this CTA's
-// tile row r, loaded ahead of time; false where write_update takes another path.
-template <int MODE>
+// The bf16 W row segment write_update<MODE, NC> reads for tile columns [c0, c0 + NC) of
+// this CTA's tile row r, loaded ahead of time; false where write_update takes another path.
+template <int MODE, int NC>
 __device__ __forceinline__ bool load_w_segment(const FinalParams& p, const ClassDesc& cd, const Tile& tl, int rank,
-                                               int r, int c0, uint4 (&w)[4]) {
+                                               int r, int c0, uint4 (&w)[NC / 8]) {
   const UpdMat& u = p.upd[cd.mat_base + tl.mat];
   const int R = Lay<MODE>::TM * tl.I + kBM * rank + r;
   const int C0 = Lay<MODE>::TN * tl.J + c0;
-  if (u.param == nullptr || !u.param_bf16 || !u.vec_param || R >= cd.rows || C0 + 32 > cd.cols) return false;
+  if (u.param == nullptr || !u.param_bf16 || !u.vec_param || R >= cd.rows || C0 + NC > cd.cols) return false;
   const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(u.param) +
                                                     static_cast<int64_t>(R) * u.ld_param + C0);
 #pragma unroll
-  for (int q = 0; q < 4; ++q) w[q] = src[q];
+  for (int q = 0; q < NC / 8; ++q) w[q] = src[q];
   return true;
 }
 
@@ -443,7 +446,7 @@ __device__ __forceinline__ void apply_quarter(const typename ParamsOf<MODE>::typ
   uint32_t v[32];
   tmem_ld_32x32b_x32(tcol, v);
   float x[32];
-  decode32(reinterpret_cast<const uint32_t*>(xh4), reinterpret_cast<const uint32_t*>(xl4), x);
+  decode_row<32>(reinterpret_cast<const uint32_t*>(xh4), reinterpret_cast<const uint32_t*>(xl4), x);
   tmem_wait_ld();
 #pragma unroll
   for (int j = 0; j < 32; ++j) x[j] = s * fmaf(p.a, x[j], __uint_as_float(v[j]));
@@ -458,48 +461,57 @@ __device__ __forceinline__ void apply_quarter(const typename ParamsOf<MODE>::typ
   }
 }
 
-// Staged variant of the same update: the old pair is read from the staged region (hi at
-// hib in the 128-byte swizzle, lo at lob in 64-byte-swizzled 8 KB quarter blocks); kApply
-// writes the new pair back in place (the region is then stored by TMA), kApplyLast updates
-// W and/or writes O (w_pre: this thread's W segment, loaded ahead, or nullptr).
-template <int MODE>
+template <int NC>
+__device__ __forceinline__ void tmem_ld_row(uint32_t taddr, uint32_t (&v)[NC]) {
+  if constexpr (NC == 32)
+    tmem_ld_32x32b_x32(taddr, v);
+  else
+    tmem_ld_32x32b_x16(taddr, v);
+}
+
+// Staged variant of the same update for NC (16 or 32) columns: the old pair is read from
+// the staged region (hi at hib in the 128-byte swizzle, lo at lob in 64-byte-swizzled 8 KB
+// quarter blocks); kApply writes the new pair back in place (the region is then stored by
+// TMA), kApplyLast updates W and/or writes O (w_pre: this thread's W segment, loaded
+// ahead, or nullptr).
+template <int MODE, int NC>
 __device__ __forceinline__ void apply_staged(const typename ParamsOf<MODE>::type& p, const ClassDesc& cd,
                                              const Tile& tl, int rank, int r, int c0, uint32_t tcol, uint8_t* hib,
                                              uint8_t* lob, float s, const uint4* w_pre = nullptr) {
-  uint32_t v[32];
-  tmem_ld_32x32b_x32(tcol, v);
-  uint4 xh4[4], xl4[2];
+  uint32_t v[NC];
+  tmem_ld_row<NC>(tcol, v);
+  uint4 xh4[NC / 8], xl4[NC / 16];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) xh4[q] = *reinterpret_cast<const uint4*>(hib + region_chunk(r, (c0 >> 3) + q));
-  // quarter c0 / 64 of the lo block; this thread's 32 bytes are chunks 2 h, 2 h + 1 of its row
+  for (int q = 0; q < NC / 8; ++q) xh4[q] = *reinterpret_cast<const uint4*>(hib + region_chunk(r, (c0 >> 3) + q));
+  // quarter c0 / 64 of the lo block; this thread's bytes are chunks lc .. of its row
   uint8_t* lq = lob + ((c0 >> 6) << 13);
   const int lc = (c0 & 63) >> 4;
 #pragma unroll
-  for (int q = 0; q < 2; ++q) xl4[q] = *reinterpret_cast<const uint4*>(lq + lo8_chunk(r, lc + q));
-  float x[32];
-  decode32(reinterpret_cast<const uint32_t*>(xh4), reinterpret_cast<const uint32_t*>(xl4), x);
+  for (int q = 0; q < NC / 16; ++q) xl4[q] = *reinterpret_cast<const uint4*>(lq + lo8_chunk(r, lc + q));
+  float x[NC];
+  decode_row<NC>(reinterpret_cast<const uint32_t*>(xh4), reinterpret_cast<const uint32_t*>(xl4), x);
   tmem_wait_ld();
 #pragma unroll
-  for (int j = 0; j < 32; ++j) x[j] = fmaf(p.a, x[j], __uint_as_float(v[j]));
+  for (int j = 0; j < NC; ++j) x[j] = fmaf(p.a, x[j], __uint_as_float(v[j]));
   if (s != 1.f) {  // iteration 0 only (uniform)
 #pragma unroll
-    for (int j = 0; j < 32; ++j) x[j] *= s;
+    for (int j = 0; j < NC; ++j) x[j] *= s;
   }
   if constexpr (MODE == kApply) {
-    uint32_t hb[16], lb[8];
+    uint32_t hb[NC / 2], lb[NC / 4];
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
+    for (int k = 0; k < NC / 4; ++k)
       split_hi_lo8x4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3], hb[2 * k], hb[2 * k + 1], lb[k]);
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
+    for (int q = 0; q < NC / 8; ++q)
       *reinterpret_cast<uint4*>(hib + region_chunk(r, (c0 >> 3) + q)) =
           make_uint4(hb[4 * q], hb[4 * q + 1], hb[4 * q + 2], hb[4 * q + 3]);
 #pragma unroll
-    for (int q = 0; q < 2; ++q)
+    for (int q = 0; q < NC / 16; ++q)
       *reinterpret_cast<uint4*>(lq + lo8_chunk(r, lc + q)) = make_uint4(lb[4 * q], lb[4 * q + 1], lb[4 * q + 2],
                                                                         lb[4 * q + 3]);
   } else {
-    write_update<MODE>(p, cd, tl, rank, r, c0, x, w_pre);
+    write_update<MODE, NC>(p, cd, tl, rank, r, c0, x, w_pre);
   }
 }
 
@@ -702,7 +714,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
     // quarter q of this pair's next tile, so the loads run three quarters ahead of use.
     const int ew = warp - 2;
     const int q4 = warp & 3;  // TMEM lanes 32 q4 .. 32 q4 + 31 belong to this warp
-    const int h = ew >> 2;    // which 32 columns of each quarter
+    constexpr int NCW = 256 / L::NEPI;  // columns of each quarter per thread (16 with 16 warps)
+    const int h = ew >> 2;              // which NCW columns of each quarter
     const int r = q4 * 32 + lane;
     const bool leader = threadIdx.x == 64;  // also the thread that waits on the barriers
     const uint32_t tempty0 = map_to_rank(smem_u32(tempty), 0);
@@ -737,9 +750,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
       const uint32_t tacc = tmem_base + static_cast<uint32_t>(acc * L::TN) + (static_cast<uint32_t>(q4 * 32) << 16);
       // kApplyLast: this thread's bf16 W segment for the quarter after the one being
       // computed is loaded one quarter ahead (the first before the accumulator wait)
-      uint4 wq[4];
+      uint4 wq[NCW / 8];
       bool wq_ok = false;
-      if constexpr (MODE == kApplyLast) wq_ok = load_w_segment<MODE>(p, cd, tl, rank, r, 32 * h, wq);
+      if constexpr (MODE == kApplyLast) wq_ok = load_w_segment<MODE, NCW>(p, cd, tl, rank, r, NCW * h, wq);
 #pragma unroll 1
       for (int q = 0; q < 4; ++q) {
         // One warp waits (for the accumulator first, then for the inputs: kApply one
@@ -779,16 +792,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
             }
           }
         }
-        const int c0 = 64 * q + 32 * h;
+        const int c0 = 64 * q + NCW * h;
         if constexpr (MODE == kApplyLast) {
-          uint4 wn[4];
-          const bool wn_ok = q < 3 && load_w_segment<MODE>(p, cd, tl, rank, r, c0 + 64, wn);
-          apply_staged<MODE>(p, cd, tl, rank, r, c0, tacc + c0, hib, lob, sc, wq_ok ? wq : nullptr);
+          uint4 wn[NCW / 8];
+          const bool wn_ok = q < 3 && load_w_segment<MODE, NCW>(p, cd, tl, rank, r, c0 + 64, wn);
+          apply_staged<MODE, NCW>(p, cd, tl, rank, r, c0, tacc + c0, hib, lob, sc, wq_ok ? wq : nullptr);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) wq[i] = wn[i];
+          for (int i = 0; i < NCW / 8; ++i) wq[i] = wn[i];
           wq_ok = wn_ok;
         } else {
-          apply_staged<MODE>(p, cd, tl, rank, r, c0, tacc + c0, hib, lob, sc);
+          apply_staged<MODE, NCW>(p, cd, tl, rank, r, c0, tacc + c0, hib, lob, sc);
         }
         if (q == 3) {
           tc_fence_before();
