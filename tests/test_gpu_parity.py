@@ -296,3 +296,24 @@ def test_full_step_streamed_variant(shape, dtype):
     else:
         W_from_O = oracle.parameter_update(W, to_np(O), w.lr, w.weight_decay, scale)
         assert rel_fro(to_np(Wt), W_from_O) <= TOL_F32
+
+
+def test_wide_4096_shapes_at_full_size_in_one_grouped_call():
+    """One matrix of each shape of the 4096-wide set (4096^2, 4096 x 14336, 14336 x 4096)
+    at full size in one grouped call -- the shape classes of the set's waves, streamed
+    variant -- against the fp64 oracle on the host."""
+    require_gpu()
+    import time
+
+    from newton_schulz_11_b200 import api
+
+    w = inputs.WORKLOADS["wide-4096-192-matrices"]
+    idx = [0, 4, 5]  # the first matrix of each shape in the layer pattern
+    Gs = [inputs.grad_np(w, 1, i) for i in idx]
+    outs = api.newton_schulz([torch.from_numpy(G).cuda() for G in Gs], coeffs=QUINTIC5)
+    for i, G, O in zip(idx, Gs, outs):
+        t0 = time.perf_counter()
+        ref = oracle.newton_schulz(G.astype(np.float64), QUINTIC5)
+        err = rel_fro(to_np(O), ref)
+        print(f"NS {w.shapes[i]}: rel err {err:.3e} (oracle {time.perf_counter() - t0:.1f} s)")
+        assert err <= TOL_O, (w.shapes[i], err)
