@@ -273,6 +273,9 @@ class PreparedMuonStep:
         check(lib().muon_workspace_size(self._arr, self._n, ctypes.byref(need)), "muon_workspace_size")
         self._ws = workspace or default_workspace(self.device)
         self._ptr, size = self._ws.ensure(int(need.value), _stream_handle(self.device, None))
+        # the buffer this step was prepared on stays alive even if the shared workspace is
+        # later grown (and its old buffer dropped) for a larger step
+        self._buf = self._ws.buf
         self._bytes = min(size, int(need.value))
         self._hyper = (float(lr), float(beta), float(weight_decay), 1 if nesterov else 0)
         self._eps = float(eps)
@@ -288,6 +291,14 @@ class PreparedMuonStep:
     @property
     def workspace(self) -> Workspace:
         return self._ws
+
+    def device_status(self, stream=None) -> Tuple[int, int]:
+        """(code, where) of the device-side status word in this step's own workspace buffer
+        (synchronises the stream)."""
+        code, where = ctypes.c_int32(0), ctypes.c_int32(0)
+        check(lib().muon_device_status(self._ptr, _stream_handle(self.device, stream), ctypes.byref(code),
+                                       ctypes.byref(where)), "muon_device_status")
+        return int(code.value), int(where.value)
 
 
 class PreparedAdamW:

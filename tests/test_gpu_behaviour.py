@@ -166,9 +166,10 @@ def test_prepared_calls_match_one_shot_calls():
         assert torch.equal(a, b)
 
 
-def test_sharded_muon_on_one_rank_is_the_plain_step():
+@pytest.mark.parametrize("waves", [1, 2])
+def test_sharded_muon_on_one_rank_is_the_plain_step(waves):
     """Without a process group (one rank) the sharded step owns every matrix and runs the
-    library's grouped step: bit-identical to muon_step."""
+    library's grouped step, one prepared step per wave: bit-identical to muon_step."""
     require_gpu()
     from newton_schulz_11_b200 import api
     from newton_schulz_11_b200.distributed import ShardedMuon
@@ -177,6 +178,37 @@ def test_sharded_muon_on_one_rank_is_the_plain_step():
     W1, m1 = _clone(Ws), _clone(ms)
     W2, m2 = _clone(Ws), _clone(ms)
     api.muon_step(W1, gs, m1, lr=0.02, weight_decay=0.01)
-    ShardedMuon(W2, gs, m2, lr=0.02, weight_decay=0.01)()
+    sh = ShardedMuon(W2, gs, m2, lr=0.02, weight_decay=0.01, waves=waves)
+    assert sh.waves == waves and sorted(i for w in sh.wave_idx for i in w) == list(range(len(gs)))
+    sh()
     for a, b in zip(W1 + m1, W2 + m2):
         assert torch.equal(a, b)
+
+
+def test_prepared_step_survives_workspace_growth():
+    """A prepared step keeps the buffer it was prepared on: growing the shared workspace for a
+    larger step afterwards (which drops the old buffer) leaves the first step's results
+    bit-identical to the plain call, and its status word readable."""
+    require_gpu()
+    from newton_schulz_11_b200 import _lib, api
+
+    Ws, gs, ms = _set(SHAPES[:2])
+    W1, m1, W2, m2 = _clone(Ws), _clone(ms), _clone(Ws), _clone(ms)
+    ws = api.Workspace(gs[0].device)
+    small = api.PreparedMuonStep(W2, gs, m2, lr=0.02, workspace=ws)
+    before = ws.nbytes
+    BW, bg, bm = _set([(1024, 2048)], seed=3)
+    big = api.PreparedMuonStep(BW, bg, bm, lr=0.02, workspace=ws)
+    assert ws.nbytes > before
+    # reuse the freed memory for something else before the small step runs again
+    junk = [torch.full((before // 4,), float("nan"), device=gs[0].device) for _ in range(2)]
+    for _ in range(2):
+        api.muon_step(W1, gs, m1, lr=0.02)
+        small()
+        big()
+    torch.cuda.synchronize()
+    del junk
+    for a, b in zip(W1 + m1, W2 + m2):
+        assert torch.equal(a, b)
+    assert small.device_status() == (_lib.MUON_OK, 0)
+    assert big.device_status() == (_lib.MUON_OK, 0)
