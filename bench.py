@@ -37,11 +37,11 @@ KINDS = ("momentum", "norm", "gram", "poly", "apply", "apply_last")
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture of
 # the benchmarked workload, keyed by kernel kind; valid only while the kernel sources hash to
 # `source_hash` (see profiles/).  Filled in from the committed ncu summary.
-NCU_TRAFFIC = {"source_hash": "cb211889b266f68e", "workload": DEFAULT_WORKLOAD,
-               "bytes_per_launch": {"momentum": 1302197504, "norm": 29952, "gram": 210061000,
-                                    "poly": 126210000, "apply": 712098000, "apply_last": 744524288}}
+NCU_TRAFFIC = {"source_hash": "33a1c5767b1496f5", "workload": DEFAULT_WORKLOAD,
+               "bytes_per_launch": {"momentum": 1217341184, "norm": 29952, "gram": 211513753,
+                                    "poly": 125891481, "apply": 548082112, "apply_last": 653104128}}
 # the same for the AdamW path (workload gpt2-124m-adamw-params, one launch per step)
-NCU_TRAFFIC_ADAMW = {"source_hash": "cb211889b266f68e", "bytes_per_launch": 893366784}
+NCU_TRAFFIC_ADAMW = {"source_hash": "33a1c5767b1496f5", "bytes_per_launch": 893594368}
 
 
 def kernel_source_hash() -> str:
