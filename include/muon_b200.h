@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define MUON_ABI_VERSION 2
+#define MUON_ABI_VERSION 3
 #define MUON_MAX_NS_STEPS 16
 
 typedef enum {
@@ -95,14 +95,15 @@ typedef struct {
 /*
  * Where one matrix's scratch lives inside the workspace (diagnostics and tests).
  * X is carried between iterations as hi + lo: hi = bf16(x) (the tensor-core operand) and
- * lo = x - hi as a signed 8-bit fixed-point residual in units of 2^(e - 15), with e the
- * exponent of hi (|x - hi| <= 2^(e - 8), so |lo| <= 127 after rounding to nearest even
- * and clamping); x = hi + lo * 2^(e - 15), and lo = 0 where hi's biased exponent is
- * below 16.
+ * lo = one byte per element holding the residual x - hi in fixed point.  With E' the
+ * biased exponent of hi raised to at least 14 and e' = E' - 127, the residual is the
+ * integer k = round-half-even((x - hi) * 2^(14 - e')), |k| <= 64 since
+ * |x - hi| <= 2^(e - 8), and the stored byte is k + 64 (0 .. 128, unsigned); then
+ * x = hi + k * 2^(e' - 14), within 2^(e - 15) of the fp32 value.
  */
 typedef struct {
   uint64_t x_hi_offset[2];   /* bf16 [rows x x_ld]: ping-pong high parts of X */
-  uint64_t x_lo_offset;      /* int8 [rows x x_lo_ld]: low part of X, see above */
+  uint64_t x_lo_offset;      /* uint8 [rows x x_lo_ld]: low part of X, see above */
   uint64_t a_offset;         /* bf16 [m x a_ld]: A = X X^T of the latest iteration */
   uint64_t b_offset;         /* bf16 [m x a_ld]: B = b A + c A A of the latest iteration */
   uint64_t scale_offset;     /* fp32: 1 / (||u||_F + eps) */

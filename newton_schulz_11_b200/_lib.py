@@ -8,6 +8,7 @@ import threading
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libmuon_b200.so")
 
+MUON_ABI_VERSION = 3  # the version of include/muon_b200.h these bindings follow
 MUON_OK = 0
 MUON_ERR_INVALID_ARG = 1
 MUON_ERR_ALIGNMENT = 2
@@ -120,6 +121,9 @@ def lib() -> ctypes.CDLL:
             raise MuonLibraryError(f"cannot load {LIB_PATH}: {e}") from e
         P = ctypes.POINTER
         h.muon_abi_version.restype = ctypes.c_int
+        if h.muon_abi_version() != MUON_ABI_VERSION:
+            raise MuonLibraryError(f"{LIB_PATH} implements ABI version {h.muon_abi_version()}, these bindings "
+                                   f"version {MUON_ABI_VERSION}; rebuild with `python -m newton_schulz_11_b200.build`")
         h.muon_status_str.restype = ctypes.c_char_p
         h.muon_status_str.argtypes = [ctypes.c_int]
         h.muon_workspace_size.restype = ctypes.c_int

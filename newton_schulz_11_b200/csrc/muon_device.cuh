@@ -371,64 +371,50 @@ __device__ __forceinline__ uint32_t float_to_bf16_bits(float x) {
   return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(x)));
 }
 
-// Splits x into hi = bf16(x) and lo = bf16(x - hi); hi + lo carries ~16 significant bits.
-__device__ __forceinline__ void split_hi_lo(float x, uint32_t& hi, uint32_t& lo) {
-  hi = float_to_bf16_bits(x);
-  lo = float_to_bf16_bits(x - bf16_bits_to_float(hi));
-}
-
-// Two values at once: hi = bf16x2 (x0 in the low half, x1 in the high half) and lo = the
-// bf16x2 of the residuals.  Same roundings as split_hi_lo element by element.
-__device__ __forceinline__ void split_hi_lo2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
-  hi = *reinterpret_cast<const uint32_t*>(&h);
-  const __nv_bfloat162 l =
-      __floats2bfloat162_rn(x0 - __uint_as_float(hi << 16), x1 - __uint_as_float(hi & 0xFFFF0000u));
-  lo = *reinterpret_cast<const uint32_t*>(&l);
-}
-
 // ---- X as hi + lo with an 8-bit lo
-// hi = bf16(x); lo = x - hi as a signed fixed-point residual in units of 2^(e - 15), e the
-// exponent of hi: |x - hi| <= 2^(e - 8) gives |lo| <= 128, rounded to nearest even and
-// clamped to [-127, 127]; x = hi + lo * 2^(e - 15).  The worst-case residual error,
-// 2^(e - 16), is the same as that of a bf16 residual.  Where hi's biased exponent is below
-// 16 (|x| < 2^-111) lo is 0.
+// hi = bf16(x).  With E' = max(biased exponent of hi, 14) and e' = E' - 127, the residual
+// x - hi is kept as the integer k = round-half-even((x - hi) 2^(14 - e')), stored as the
+// byte k + 64, and x = hi + k 2^(e' - 14).  |x - hi| <= 2^(e - 8) bounds |k| by 64, so k
+// needs no clamp, and the residual error is at most 2^(e - 15): 15 significant bits in
+// all.  The helpers use one fma each way and byte permutes; the only integer arithmetic is
+// the exponent mask, its clamp and one subtraction.
 
-// 2^(e - 15) for the bf16 hi (bit pattern in the low 16 bits), or 0 (integer exponent
-// arithmetic only).
-__device__ __forceinline__ float lo8_unit(uint32_t hi16) {
-  const int32_t eb = static_cast<int32_t>((hi16 << 16) & 0x7F800000u);
-  return __int_as_float(max(eb - (15 << 23), 0));
+// 2^e' as float bits, from hi's float bits hb.
+__device__ __forceinline__ uint32_t lo8_exp_bits(uint32_t hb) { return max(hb & 0x7F800000u, 14u << 23); }
+
+// The stored byte for x against hi (float bits hb), in the low 8 bits of the result (the
+// bits above belong to 1.5 * 2^23 and are dropped by the caller): one fma scales the exact
+// residual by 2^(14 - e') (float bits 0x86000000 - 2^e' bits), rounds it to the nearest
+// integer, ties to even, and adds 1.5 * 2^23 + 64.
+__device__ __forceinline__ uint32_t lo8_encode_word(float x, uint32_t hb) {
+  const float r = x - __uint_as_float(hb);  // exact
+  return __float_as_uint(fmaf(r, __uint_as_float(0x86000000u - lo8_exp_bits(hb)), 12582976.f));
 }
 
-// The 8-bit residual of x against its bf16 hi (bit pattern hi16), as a byte.  The scaled
-// residual is clamped, then rounded to nearest even by adding 1.5 * 2^23, which leaves the
-// integer's two's complement in the low bits of the sum (full-rate float and integer ops).
+// The stored byte for x against the bf16 hi (bit pattern in the low 16 bits).
 __device__ __forceinline__ uint32_t lo8_encode(float x, uint32_t hi16) {
-  const uint32_t hb = hi16 << 16;
-  const uint32_t eb = hb & 0x7F800000u;
-  const float r = x - __uint_as_float(hb);                                   // exact
-  const float t = fminf(fmaxf(r * __uint_as_float(0x86800000u - eb), -127.f), 127.f);  // r * 2^(15 - e)
-  const uint32_t q = __float_as_uint(t + 12582912.f) & 0xFFu;
-  return eb >= (16u << 23) ? q : 0u;
+  return lo8_encode_word(x, hi16 << 16) & 0xFFu;
 }
 
-// x from a bf16 hi (bits hi16) and its 8-bit residual (byte lo8).
-__device__ __forceinline__ float lo8_decode(uint32_t hi16, uint32_t lo8) {
-  const uint32_t k = static_cast<uint32_t>(static_cast<int32_t>(lo8 << 24) >> 24);  // sign-extended
-  const float q = __uint_as_float(0x4B400000u + k) - 12582912.f;
-  return fmaf(q, lo8_unit(hi16), __uint_as_float(hi16 << 16));
+// x from hi (float bits hb) and the stored byte j (0..3) of word lw: a byte permute makes
+// the float 1.5 * 2^23 + byte, one fma turns it into k 2^-14 (exact), one more adds
+// k 2^(e' - 14) to hi.
+__device__ __forceinline__ float lo8_decode(uint32_t hb, uint32_t lw, uint32_t j) {
+  const float f = __uint_as_float(__byte_perm(lw, 0x4B400000u, 0x7650u | j));
+  const float k = fmaf(f, 0x1p-14f, -768.00390625f);  // (f - 1.5 * 2^23 - 64) * 2^-14
+  return fmaf(k, __uint_as_float(lo8_exp_bits(hb)), __uint_as_float(hb));
 }
 
 // Four values at once: hi as two bf16x2 words (h01: x0 low, x1 high; h23 likewise) and the
-// four residual bytes in one word (x0 in the lowest byte).
+// four stored bytes in one word (x0 in the lowest byte).
 __device__ __forceinline__ void split_hi_lo8x4(float x0, float x1, float x2, float x3, uint32_t& h01, uint32_t& h23,
                                                uint32_t& l4) {
   const __nv_bfloat162 a = __floats2bfloat162_rn(x0, x1), b = __floats2bfloat162_rn(x2, x3);
   h01 = *reinterpret_cast<const uint32_t*>(&a);
   h23 = *reinterpret_cast<const uint32_t*>(&b);
-  l4 = lo8_encode(x0, h01 & 0xFFFFu) | (lo8_encode(x1, h01 >> 16) << 8) | (lo8_encode(x2, h23 & 0xFFFFu) << 16) |
-       (lo8_encode(x3, h23 >> 16) << 24);
+  const uint32_t w0 = lo8_encode_word(x0, h01 << 16), w1 = lo8_encode_word(x1, h01 & 0xFFFF0000u);
+  const uint32_t w2 = lo8_encode_word(x2, h23 << 16), w3 = lo8_encode_word(x3, h23 & 0xFFFF0000u);
+  l4 = __byte_perm(__byte_perm(w0, w1, 0x0040u), __byte_perm(w2, w3, 0x0040u), 0x5410u);
 }
 
 // L2 prefetch of the line holding `p`.

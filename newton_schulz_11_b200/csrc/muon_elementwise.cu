@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(kEwThreads) muon_momentum_kernel(const __grid_
       if (!ns_only) *mp = m;
       const uint32_t h = float_to_bf16_bits(u);
       t.hi[static_cast<int64_t>(r) * t.ldx + c] = __ushort_as_bfloat16(static_cast<unsigned short>(h));
-      t.lo[static_cast<int64_t>(r) * t.ldl + c] = static_cast<int8_t>(lo8_encode(u, h));
+      t.lo[static_cast<int64_t>(r) * t.ldl + c] = static_cast<uint8_t>(lo8_encode(u, h));
       acc = fmaf(u, u, acc);
     }
   }

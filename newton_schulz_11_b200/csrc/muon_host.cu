@@ -401,7 +401,7 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
     const int count = static_cast<int>(c.mats.size());
     __nv_bfloat16* hi0 = reinterpret_cast<__nv_bfloat16*>(ws + c.off_hi[0]);
     __nv_bfloat16* hi1 = reinterpret_cast<__nv_bfloat16*>(ws + c.off_hi[1]);
-    int8_t* lo = reinterpret_cast<int8_t*>(ws + c.off_lo);
+    uint8_t* lo = reinterpret_cast<uint8_t*>(ws + c.off_lo);
     __nv_bfloat16* ab = reinterpret_cast<__nv_bfloat16*>(ws + c.off_a);
     __nv_bfloat16* bb = reinterpret_cast<__nv_bfloat16*>(ws + c.off_b);
     if (!encode_map(&op_hi[ci][0], hi0, count, c.rows, c.cols, c.ldx, 128) ||

@@ -256,23 +256,25 @@ __device__ __forceinline__ void load_row32(const __nv_bfloat16* row, int valid, 
   }
 }
 
-// 32 consecutive bytes of a row of the 8-bit lo buffer (two 16-byte loads), zero past
-// `valid` columns or when `live` is false.  `row` is 16-byte aligned.
-__device__ __forceinline__ void load_row32_u8(const int8_t* row, int valid, bool live, uint4 (&w)[2]) {
+// 32 consecutive bytes of a row of the 8-bit lo buffer (two 16-byte loads); past `valid`
+// columns, or when `live` is false, the byte of a zero residual (0x40).  `row` is 16-byte
+// aligned.
+__device__ __forceinline__ void load_row32_u8(const uint8_t* row, int valid, bool live, uint4 (&w)[2]) {
+  constexpr uint32_t kZero4 = 0x40404040u;
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
     if (live && 16 * q < valid)
       w[q] = __ldg(reinterpret_cast<const uint4*>(row) + q);
     else
-      w[q] = make_uint4(0u, 0u, 0u, 0u);
+      w[q] = make_uint4(kZero4, kZero4, kZero4, kZero4);
   }
   if (live && valid < 32 && valid > 0) {
     uint32_t* e = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int k = valid - 4 * j;  // bytes of word j that lie inside the row
-      if (k <= 0) e[j] = 0u;
-      else if (k < 4) e[j] &= (1u << (8 * k)) - 1u;
+      if (k <= 0) e[j] = kZero4;
+      else if (k < 4) e[j] = (e[j] & ((1u << (8 * k)) - 1u)) | (kZero4 & ~((1u << (8 * k)) - 1u));
     }
   }
 }
@@ -285,16 +287,16 @@ __device__ __forceinline__ uint32_t lo8_chunk(int r, int c) {
   return static_cast<uint32_t>(r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
 }
 
-// Decodes NC values of a row: x_j = hi_j + lo_j 2^(e_j - 15) for the bf16 pairs in `h`
-// (NC / 2 words, element 2i in the low half of word i) and the residual bytes in `l`
-// (NC / 4 words, element j in byte j % 4 of word j / 4).
+// Decodes NC values of a row from their bf16 hi and 8-bit lo: the bf16 pairs in `h`
+// (NC / 2 words, element 2i in the low half of word i) and the stored residual bytes in
+// `l` (NC / 4 words, element j in byte j % 4 of word j / 4).
 template <int NC>
 __device__ __forceinline__ void decode_row(const uint32_t* h, const uint32_t* l, float (&x)[NC]) {
 #pragma unroll
   for (int i = 0; i < NC / 2; ++i) {
-    const uint32_t lw = l[i >> 1] >> (16 * (i & 1));
-    x[2 * i] = lo8_decode(h[i] & 0xFFFFu, lw & 0xFFu);
-    x[2 * i + 1] = lo8_decode(h[i] >> 16, (lw >> 8) & 0xFFu);
+    const uint32_t j = 2u * static_cast<uint32_t>(i & 1);
+    x[2 * i] = lo8_decode(h[i] << 16, l[i >> 1], j);
+    x[2 * i + 1] = lo8_decode(h[i] & 0xFFFF0000u, l[i >> 1], j + 1u);
   }
 }
 

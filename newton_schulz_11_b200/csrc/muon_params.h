@@ -58,7 +58,7 @@ struct ClassDesc {
   int32_t pad_;
   __nv_bfloat16* x_hi_cur;   // hi part read this iteration
   __nv_bfloat16* x_hi_next;  // hi part written this iteration
-  int8_t* x_lo;              // lo part (8-bit residual of hi), updated in place
+  uint8_t* x_lo;             // lo part (stored 8-bit residual of hi), updated in place
   __nv_bfloat16* a_buf;
   __nv_bfloat16* b_buf;
 };
@@ -101,7 +101,7 @@ struct EwMat {
   const float* g;
   float* m;
   __nv_bfloat16* hi;
-  int8_t* lo;               // 8-bit residual of hi, row stride ldl bytes
+  uint8_t* lo;              // stored 8-bit residual of hi, row stride ldl bytes
   int64_t ld_g, ld_m;
   int32_t rows, cols, ldx, ldl;
   int32_t rows_per_chunk;

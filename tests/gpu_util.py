@@ -27,21 +27,21 @@ def ws_matrix(ws_buf, offset, rows, cols, ld, dtype=torch.bfloat16):
 
 
 def lo8_unit(hi):
-    """2^(e - 15) per element for a bf16-valued tensor hi (e its exponent), 0 where the biased
-    exponent is below 16 -- the unit of the 8-bit lo part (include/muon_b200.h)."""
+    """2^(e' - 14) per element for a bf16-valued tensor hi, with e' its exponent raised to at
+    least -113 (biased 14) -- the unit of the 8-bit lo part (include/muon_b200.h)."""
     E = (hi.float().contiguous().view(torch.int32) >> 23) & 0xFF
-    # built from exponent bits: exactly 2^(e - 15) (a pow() may be off in the last bit,
+    # built from exponent bits: exactly 2^(e' - 14) (a pow() may be off in the last bit,
     # which moves exact ties of the rounding)
-    unit = (((E - 15).clamp(min=1)) << 23).to(torch.int32).view(torch.float32).double()
-    return torch.where(E >= 16, unit, torch.zeros_like(unit))
+    return ((E.clamp(min=14) - 14) << 23).to(torch.int32).view(torch.float32).double().where(
+        E > 14, torch.full_like(E, 2.0 ** -127, dtype=torch.float64))
 
 
 def ws_lo8(ws_buf, offset, rows, cols, ld_bytes, hi):
-    """The 8-bit lo part of X inside the workspace, as fp64 values (q * 2^(e - 15)), and the
-    raw signed bytes q."""
-    raw = ws_buf[offset: offset + rows * ld_bytes].view(torch.int8).reshape(rows, ld_bytes)[:, :cols]
-    q = raw.double()
-    return q * lo8_unit(hi), q
+    """The 8-bit lo part of X inside the workspace, as fp64 values (k * 2^(e' - 14)), and the
+    residual integers k (stored byte - 64)."""
+    raw = ws_buf[offset: offset + rows * ld_bytes].view(torch.uint8).reshape(rows, ld_bytes)[:, :cols]
+    k = raw.double() - 64.0
+    return k * lo8_unit(hi), k
 
 
 def ws_scalar(ws_buf, offset):

@@ -38,7 +38,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.muon_abi_version() == 2
+    assert L.muon_abi_version() == _lib.MUON_ABI_VERSION == 3
     for code in range(9):
         assert L.muon_status_str(code).decode() not in ("", "unknown status")
     assert L.muon_status_str(99).decode() == "unknown status"
