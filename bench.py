@@ -37,11 +37,11 @@ KINDS = ("momentum", "norm", "gram", "poly", "apply", "apply_last")
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture of
 # the benchmarked workload, keyed by kernel kind; valid only while the kernel sources hash to
 # `source_hash` (see profiles/).  Filled in from the committed ncu summary.
-NCU_TRAFFIC = {"source_hash": "33a1c5767b1496f5", "workload": DEFAULT_WORKLOAD,
-               "bytes_per_launch": {"momentum": 1217341184, "norm": 29952, "gram": 211513753,
-                                    "poly": 125891481, "apply": 548082112, "apply_last": 653104128}}
+NCU_TRAFFIC = {"source_hash": "be70e1446178eb8e", "workload": DEFAULT_WORKLOAD,
+               "bytes_per_launch": {"momentum": 1218154240, "norm": 29696, "gram": 209802752,
+                                    "poly": 126076416, "apply": 549483200, "apply_last": 652814336}}
 # the same for the AdamW path (workload gpt2-124m-adamw-params, one launch per step)
-NCU_TRAFFIC_ADAMW = {"source_hash": "33a1c5767b1496f5", "bytes_per_launch": 893594368}
+NCU_TRAFFIC_ADAMW = {"source_hash": "be70e1446178eb8e", "bytes_per_launch": 893892096}
 
 
 def kernel_source_hash() -> str:
