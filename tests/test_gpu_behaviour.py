@@ -212,3 +212,29 @@ def test_prepared_step_survives_workspace_growth():
         assert torch.equal(a, b)
     assert small.device_status() == (_lib.MUON_OK, 0)
     assert big.device_status() == (_lib.MUON_OK, 0)
+
+
+def test_step_replays_from_a_cuda_graph():
+    """A step is kernel launches only (parameters by value, no host copies or syncs), so it
+    can be captured in a CUDA graph; each replay equals an eager step bit for bit."""
+    require_gpu()
+    from newton_schulz_11_b200 import _lib, api
+
+    Ws, gs, ms = _set(SHAPES)
+    W1, m1, W2, m2 = _clone(Ws), _clone(ms), _clone(Ws), _clone(ms)
+    eager = api.PreparedMuonStep(W1, gs, m1, lr=0.02, weight_decay=0.01)
+    graphed = api.PreparedMuonStep(W2, gs, m2, lr=0.02, weight_decay=0.01)
+    eager()
+    graphed()  # the first call builds and caches the host-side plan
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        graphed()
+    for _ in range(3):
+        eager()
+        g.replay()
+        torch.cuda.synchronize()
+        for a, b in zip(W1 + m1, W2 + m2):
+            assert torch.equal(a, b)
+    assert graphed.device_status() == (_lib.MUON_OK, 0)
+    del g
