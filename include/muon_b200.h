@@ -32,7 +32,10 @@
  * Execution: asynchronous on `stream` (a cudaStream_t; NULL is the legacy default
  * stream).  No call synchronises the host except muon_device_status.  The first
  * call with a new set of descriptors plans the work (host only, microseconds) and
- * caches the plan; later calls with identical descriptors reuse it.
+ * caches the plan; later calls with identical descriptors reuse it.  muon_step and
+ * muon_newton_schulz queue kernel launches only (arguments by value, no copies, no
+ * host synchronisation), so they can be captured in a CUDA graph; every buffer and
+ * the workspace must then stay in place for as long as the graph is replayed.
  *
  * Errors: every entry point returns a muon_status_t.  On a validation error
  * nothing is launched and no buffer is touched.  A failed CUDA launch returns
@@ -41,9 +44,10 @@
  * muon_device_status) and the kernel returns instead of hanging.
  *
  * Numerics: Newton-Schulz runs with bf16 tensor-core operands and fp32
- * accumulation; X is carried between iterations as a bf16 pair (hi + lo), which
- * holds about 16 significant bits, so that the a*X term does not lose the
- * precision a single bf16 copy would.  Momentum and the update are fp32.
+ * accumulation; X is carried between iterations as a bf16 hi plus an 8-bit
+ * fixed-point residual (15 significant bits, see muon_scratch_view_t), so that the
+ * a*X term does not lose the precision a single bf16 copy would.  Momentum and the
+ * update are fp32.
  * Finite inputs with ||u||_F below about 1e17 are required (the Gram of the
  * unscaled bf16 input is formed before the 1/||u||^2 factor is applied).
  */
@@ -230,7 +234,7 @@ muon_status_t muon_adamw_step(const muon_adamw_tensor_t* tensors, int n, float l
  * device memory: code that runs inside another framework's memory pool or allocator
  * (where a cudaMalloc of its own would fragment that pool, or is forbidden), plugins
  * and embedded hosts that only receive ready-made device buffers, and callers that
- * must not allocate between steps.  There is no counterpart in the paper; this is a
+ * must not allocate between steps.  The pages define no such call; this is a
  * packaging of muon_newton_schulz.
  *
  * Same arguments and results as muon_newton_schulz, except that the scratch is a
