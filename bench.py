@@ -36,20 +36,47 @@ KINDS = ("momentum", "norm", "gram", "poly", "apply", "apply_last")
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture of
 # the benchmarked workload, keyed by kernel kind; valid only while the kernel sources hash to
-# `source_hash` (see profiles/).  Filled in from the committed ncu summary.
-NCU_TRAFFIC = {"source_hash": "be70e1446178eb8e", "workload": DEFAULT_WORKLOAD,
+# `source_hash` (kernel_source_hash: comments and layout do not count; see profiles/).
+# Filled in from the committed ncu summary.
+NCU_TRAFFIC = {"source_hash": "2854712ec87fa922", "workload": DEFAULT_WORKLOAD,
                "bytes_per_launch": {"momentum": 1218154240, "norm": 29696, "gram": 209802752,
                                     "poly": 126076416, "apply": 549483200, "apply_last": 652814336}}
 # the same for the AdamW path (workload gpt2-124m-adamw-params, one launch per step)
-NCU_TRAFFIC_ADAMW = {"source_hash": "be70e1446178eb8e", "bytes_per_launch": 893892096}
+NCU_TRAFFIC_ADAMW = {"source_hash": "2854712ec87fa922", "bytes_per_launch": 893892096}
+
+
+def _code_only(text: str) -> str:
+    """C/C++/CUDA source with comments removed and whitespace runs collapsed: what the
+    compiler sees, so that an edit to a comment does not invalidate measured counters."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":  # string or character literal, copied through with its escapes
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
 
 
 def kernel_source_hash() -> str:
+    """Hash of the kernel sources (newton_schulz_11_b200/csrc), comments and layout aside."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "newton_schulz_11_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(name.encode() + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

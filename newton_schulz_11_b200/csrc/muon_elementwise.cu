@@ -2,8 +2,9 @@
 //
 //   m' = beta m + g                        ("14 - modded-nanogpt", section 3, muon_step)
 //   u  = g + beta m'  (Nesterov) or m'     ("NanoGPT Speedrun" README, practices list)
-//   hi = bf16(u), lo = 8-bit residual      Newton-Schulz input, unscaled (lo in units of
-//                                          2^(e - 15), e the exponent of hi)
+//   hi = bf16(u), lo = 8-bit residual      Newton-Schulz input, unscaled (lo: the byte
+//                                          k + 64, k the residual in units of 2^(e' - 14),
+//                                          e' the exponent of hi raised to at least -113)
 //   partial[chunk] = sum of u^2            for ||u||_F of the listing's G.norm()
 //
 // followed by a per-matrix finalisation s = 1 / (||u||_F + eps) in a fixed order
