@@ -317,3 +317,46 @@ def test_wide_4096_shapes_at_full_size_in_one_grouped_call():
         err = rel_fro(to_np(O), ref)
         print(f"NS {w.shapes[i]}: rel err {err:.3e} (oracle {time.perf_counter() - t0:.1f} s)")
         assert err <= TOL_O, (w.shapes[i], err)
+
+
+def test_bf16_update_on_ragged_views_keeps_the_neighbours():
+    """The last apply stores a bf16 W tile through its staging by TMA when W's rows are
+    16-byte aligned, and element by element otherwise.  Ragged shapes as strided views
+    inside larger sentinel-filled buffers, both kinds in one grouped call: W within one
+    bf16 ulp of the oracle's update of the GPU's own O, O against the oracle, and every
+    element outside the views untouched."""
+    require_gpu()
+    from newton_schulz_11_b200 import api
+
+    # (rows, cols, column offset of the view in elements): offset 8 keeps 16-byte rows
+    # (tensor-map path), offset 4 does not (element path)
+    cases = [(136, 200, 8), (200, 136, 8), (72, 40, 8), (264, 776, 8), (128, 384, 8), (136, 200, 4)]
+    lr, wd, beta = 0.02, 0.01, 0.95
+    rng = np.random.default_rng(11)
+    bufs, Ws, gs, ms, outs, W_in, g_in, m_in = [], [], [], [], [], [], [], []
+    for r, c, off in cases:
+        buf = torch.full((r + 3, c + 24), 7.0, dtype=torch.bfloat16, device="cuda")
+        W = buf[1:1 + r, off:off + c]
+        W.copy_(torch.from_numpy(rng.standard_normal((r, c)) * 0.02).to(torch.bfloat16))
+        g = rng.standard_normal((r, c)).astype(np.float32)
+        m = rng.standard_normal((r, c)).astype(np.float32)
+        bufs.append(buf)
+        Ws.append(W)
+        gs.append(torch.from_numpy(g).cuda())
+        ms.append(torch.from_numpy(m).cuda())
+        outs.append(torch.empty((r, c), device="cuda"))
+        W_in.append(to_np(W))
+        g_in.append(g.astype(np.float64))
+        m_in.append(m.astype(np.float64))
+    api.muon_step(Ws, gs, ms, lr=lr, beta=beta, weight_decay=wd, nesterov=True, coeffs=QUINTIC5, outs=outs)
+    torch.cuda.synchronize()
+    for k, (r, c, off) in enumerate(cases):
+        m_ref = oracle.momentum_update(m_in[k], g_in[k], beta)
+        O_ref = oracle.newton_schulz(oracle.nesterov_input(g_in[k], m_ref, beta, True), QUINTIC5)
+        err = rel_fro(to_np(outs[k]), O_ref)
+        assert err <= TOL_O, f"O {r}x{c}: {err:.3e}"
+        scale = float(np.sqrt(max(1.0, r / c)))
+        check_bf16_update(to_np(Ws[k]), W_in[k], to_np(outs[k]), lr, wd, scale, f"W {r}x{c} offset {off}")
+        outside = torch.ones_like(bufs[k], dtype=torch.bool)
+        outside[1:1 + r, off:off + c] = False
+        assert bool((bufs[k][outside] == 7.0).all()), f"{r}x{c} offset {off}: an element outside the view changed"
