@@ -481,8 +481,13 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
         u.ld_param = t.ld_param;
         u.param_bf16 = t.param_dtype == MUON_BF16 ? 1 : 0;
         const int pv = u.param_bf16 ? 8 : 4;
-        u.vec_param = (t.param != nullptr && aligned(t.param, 16) && t.ld_param % pv == 0) ? 1 : 0;
-        u.vec_out = (t.out_update != nullptr && aligned(t.out_update, 16) && t.cols % 4 == 0) ? 1 : 0;
+        // 1: rows 16-byte aligned (128-bit accesses); 2: 32-byte aligned (256-bit accesses)
+        u.vec_param = (t.param != nullptr && aligned(t.param, 16) && t.ld_param % pv == 0)
+                          ? ((aligned(t.param, 32) && t.ld_param % (2 * pv) == 0) ? 2 : 1)
+                          : 0;
+        u.vec_out = (t.out_update != nullptr && aligned(t.out_update, 16) && t.cols % 4 == 0)
+                        ? ((aligned(t.out_update, 32) && t.cols % 8 == 0) ? 2 : 1)
+                        : 0;
       }
     }
   }

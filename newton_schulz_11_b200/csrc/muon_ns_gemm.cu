@@ -368,7 +368,15 @@ __device__ __forceinline__ void write_update(const FinalParams& p, const ClassDe
   const UpdMat& u = p.upd[cd.mat_base + tl.mat];
   if (u.out != nullptr) {
     float* o = u.out + static_cast<int64_t>(R) * cols + C0;
-    if (full && u.vec_out) {
+    if (full && u.vec_out == 2) {
+#pragma unroll
+      for (int q = 0; q < NC / 8; ++q)
+        st_global_v8(o + 8 * q,
+                     make_uint4(__float_as_uint(x[8 * q]), __float_as_uint(x[8 * q + 1]), __float_as_uint(x[8 * q + 2]),
+                                __float_as_uint(x[8 * q + 3])),
+                     make_uint4(__float_as_uint(x[8 * q + 4]), __float_as_uint(x[8 * q + 5]),
+                                __float_as_uint(x[8 * q + 6]), __float_as_uint(x[8 * q + 7])));
+    } else if (full && u.vec_out) {
 #pragma unroll
       for (int q = 0; q < NC / 4; ++q)
         reinterpret_cast<float4*>(o)[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
@@ -383,17 +391,33 @@ __device__ __forceinline__ void write_update(const FinalParams& p, const ClassDe
     if (u.param_bf16) {
       __nv_bfloat16* w = static_cast<__nv_bfloat16*>(u.param) + static_cast<int64_t>(R) * u.ld_param + C0;
       if (full && u.vec_param) {
+        const bool v8 = u.vec_param == 2;  // 32-byte rows: 256-bit accesses
         uint4 raw[NC / 8];
+        if (w_pre != nullptr) {
 #pragma unroll
-        for (int q = 0; q < NC / 8; ++q) raw[q] = w_pre != nullptr ? w_pre[q] : reinterpret_cast<const uint4*>(w)[q];
+          for (int q = 0; q < NC / 8; ++q) raw[q] = w_pre[q];
+        } else if (v8) {
+#pragma unroll
+          for (int q = 0; q < NC / 16; ++q) ld_global_v8(w + 16 * q, raw[2 * q], raw[2 * q + 1]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < NC / 8; ++q) raw[q] = reinterpret_cast<const uint4*>(w)[q];
+        }
         const uint32_t* rw = reinterpret_cast<const uint32_t*>(raw);
         uint32_t wb[NC / 2];
 #pragma unroll
         for (int i = 0; i < NC / 2; ++i)
           wb[i] = pack_bf16x2(fmaf(-ls, x[2 * i], lo_bf16(rw[i]) * decay), fmaf(-ls, x[2 * i + 1], hi_bf16(rw[i]) * decay));
+        if (v8) {
 #pragma unroll
-        for (int q = 0; q < NC / 8; ++q)
-          reinterpret_cast<uint4*>(w)[q] = make_uint4(wb[4 * q], wb[4 * q + 1], wb[4 * q + 2], wb[4 * q + 3]);
+          for (int q = 0; q < NC / 16; ++q)
+            st_global_v8(w + 16 * q, make_uint4(wb[8 * q], wb[8 * q + 1], wb[8 * q + 2], wb[8 * q + 3]),
+                         make_uint4(wb[8 * q + 4], wb[8 * q + 5], wb[8 * q + 6], wb[8 * q + 7]));
+        } else {
+#pragma unroll
+          for (int q = 0; q < NC / 8; ++q)
+            reinterpret_cast<uint4*>(w)[q] = make_uint4(wb[4 * q], wb[4 * q + 1], wb[4 * q + 2], wb[4 * q + 3]);
+        }
       } else {
 #pragma unroll
         for (int j = 0; j < NC; ++j)
@@ -401,7 +425,18 @@ __device__ __forceinline__ void write_update(const FinalParams& p, const ClassDe
       }
     } else {
       float* w = static_cast<float*>(u.param) + static_cast<int64_t>(R) * u.ld_param + C0;
-      if (full && u.vec_param) {
+      if (full && u.vec_param == 2) {
+#pragma unroll
+        for (int q = 0; q < NC / 8; ++q) {
+          uint4 a, b;
+          ld_global_v8(w + 8 * q, a, b);
+          const uint32_t in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+          uint32_t out[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) out[j] = __float_as_uint(fmaf(-ls, x[8 * q + j], __uint_as_float(in[j]) * decay));
+          st_global_v8(w + 8 * q, make_uint4(out[0], out[1], out[2], out[3]), make_uint4(out[4], out[5], out[6], out[7]));
+        }
+      } else if (full && u.vec_param) {
 #pragma unroll
         for (int q = 0; q < NC / 4; ++q) {
           float4 t = reinterpret_cast<float4*>(w)[q];
@@ -429,10 +464,14 @@ __device__ __forceinline__ bool load_w_segment(const FinalParams& p, const Class
   const int R = Lay<MODE>::TM * tl.I + kBM * rank + r;
   const int C0 = Lay<MODE>::TN * tl.J + c0;
   if (u.param == nullptr || !u.param_bf16 || !u.vec_param || R >= cd.rows || C0 + NC > cd.cols) return false;
-  const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(u.param) +
-                                                    static_cast<int64_t>(R) * u.ld_param + C0);
+  const __nv_bfloat16* row = static_cast<const __nv_bfloat16*>(u.param) + static_cast<int64_t>(R) * u.ld_param + C0;
+  if (u.vec_param == 2) {  // 32-byte rows: 256-bit loads
 #pragma unroll
-  for (int q = 0; q < NC / 8; ++q) w[q] = src[q];
+    for (int q = 0; q < NC / 16; ++q) ld_global_v8(row + 16 * q, w[2 * q], w[2 * q + 1]);
+  } else {
+#pragma unroll
+    for (int q = 0; q < NC / 8; ++q) w[q] = reinterpret_cast<const uint4*>(row)[q];
+  }
   return true;
 }
 

@@ -70,8 +70,8 @@ struct UpdMat {
   int64_t ld_param;
   float lr_scale;         // lr * shape_scale
   int32_t param_bf16;
-  int32_t vec_param;      // W rows are 16-byte aligned: vector stores allowed
-  int32_t vec_out;        // O rows are 16-byte aligned
+  int32_t vec_param;      // W rows 16-byte aligned (1: 128-bit accesses) or 32-byte (2: 256-bit)
+  int32_t vec_out;        // O rows likewise
 };
 
 struct GemmParams {

@@ -320,17 +320,19 @@ def test_wide_4096_shapes_at_full_size_in_one_grouped_call():
 
 
 def test_bf16_update_on_ragged_views_keeps_the_neighbours():
-    """The last apply stores a bf16 W tile through its staging by TMA when W's rows are
-    16-byte aligned, and element by element otherwise.  Ragged shapes as strided views
-    inside larger sentinel-filled buffers, both kinds in one grouped call: W within one
-    bf16 ulp of the oracle's update of the GPU's own O, O against the oracle, and every
-    element outside the views untouched."""
+    """The last apply updates bf16 W with 256-bit, 128-bit or element accesses, by the
+    alignment of W's rows.  Ragged shapes as strided views inside larger sentinel-filled
+    buffers, all three kinds in one grouped call: W within one bf16 ulp of the oracle's
+    update of the GPU's own O, O against the oracle, and every element outside the views
+    untouched."""
     require_gpu()
     from newton_schulz_11_b200 import api
 
-    # (rows, cols, column offset of the view in elements): offset 8 keeps 16-byte rows
-    # (tensor-map path), offset 4 does not (element path)
-    cases = [(136, 200, 8), (200, 136, 8), (72, 40, 8), (264, 776, 8), (128, 384, 8), (136, 200, 4)]
+    # (rows, cols, column offset of the view in elements): offset 16 keeps the rows 32-byte
+    # aligned (256-bit accesses), offset 8 16-byte aligned (128-bit), offset 4 neither
+    # (element by element)
+    cases = [(136, 200, 8), (200, 136, 8), (72, 40, 8), (264, 776, 8), (128, 384, 8), (136, 200, 4),
+             (136, 200, 16), (264, 776, 16)]
     lr, wd, beta = 0.02, 0.01, 0.95
     rng = np.random.default_rng(11)
     bufs, Ws, gs, ms, outs, W_in, g_in, m_in = [], [], [], [], [], [], [], []
