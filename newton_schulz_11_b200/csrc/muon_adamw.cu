@@ -34,7 +34,7 @@ struct AdamTensor {
   int64_t numel;
   int64_t chunk_begin;  // first chunk of this tensor in the launch
   int32_t p_bf16;
-  int32_t vec;  // 16-byte aligned g, m, v (and p: 8 bytes for bf16, 16 for fp32)
+  int32_t vec;  // 1: 16-byte aligned g, m, v (p: 8 bytes for bf16, 16 for fp32); 2: twice that
 };
 
 struct AdamParams {
@@ -69,7 +69,39 @@ __global__ void __launch_bounds__(kAdamThreads) muon_adamw_kernel(const __grid_c
   const int64_t e0 = (chunk - t.chunk_begin) * kAdamChunk;
   const int64_t e1 = t.numel < e0 + kAdamChunk ? t.numel : e0 + kAdamChunk;
   int64_t scalar_from = e0;
-  if (t.vec) {
+  if (t.vec == 2) {  // 32-byte aligned tensors: eight elements per thread and access
+    const int64_t n8 = (e1 - e0) >> 3;
+    for (int64_t i = threadIdx.x; i < n8; i += kAdamThreads) {
+      const int64_t e = e0 + 8 * i;
+      float g[8], m[8], v[8], pv[8];
+      ld_global_cs_v8(t.g + e, g);
+      ld_global_cs_v8(t.m + e, m);
+      ld_global_cs_v8(t.v + e, v);
+      if (t.p_bf16) {
+        __nv_bfloat16* pp = static_cast<__nv_bfloat16*>(t.p) + e;
+        const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(pp));
+        const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
+        uint32_t out[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float p0 = adam_one(a, bf16_bits_to_float(rw[k] & 0xFFFFu), g[2 * k], m[2 * k], v[2 * k]);
+          const float p1 = adam_one(a, bf16_bits_to_float(rw[k] >> 16), g[2 * k + 1], m[2 * k + 1], v[2 * k + 1]);
+          const __nv_bfloat162 q = __floats2bfloat162_rn(p0, p1);
+          out[k] = *reinterpret_cast<const uint32_t*>(&q);
+        }
+        __stcs(reinterpret_cast<uint4*>(pp), make_uint4(out[0], out[1], out[2], out[3]));
+      } else {
+        float* pp = static_cast<float*>(t.p) + e;
+        ld_global_cs_v8(pp, pv);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) pv[k] = adam_one(a, pv[k], g[k], m[k], v[k]);
+        st_global_cs_v8(pp, pv);
+      }
+      st_global_cs_v8(t.m + e, m);
+      st_global_cs_v8(t.v + e, v);
+    }
+    scalar_from = e0 + 8 * n8;
+  } else if (t.vec) {
     const int64_t n4 = (e1 - e0) >> 2;
     for (int64_t i = threadIdx.x; i < n4; i += kAdamThreads) {
       const int64_t e = e0 + 4 * i;
@@ -214,8 +246,11 @@ extern "C" muon_status_t muon_adamw_step(const muon_adamw_tensor_t* ts, int n, f
       d.numel = t.numel;
       d.chunk_begin = chunks;
       d.p_bf16 = t.param_dtype == MUON_BF16 ? 1 : 0;
-      d.vec = (aligned_to(t.grad, 16) && aligned_to(t.exp_avg, 16) && aligned_to(t.exp_avg_sq, 16) &&
-               aligned_to(t.param, d.p_bf16 ? 8 : 16))
+      d.vec = (aligned_to(t.grad, 32) && aligned_to(t.exp_avg, 32) && aligned_to(t.exp_avg_sq, 32) &&
+               aligned_to(t.param, d.p_bf16 ? 16 : 32))
+                  ? 2
+              : (aligned_to(t.grad, 16) && aligned_to(t.exp_avg, 16) && aligned_to(t.exp_avg_sq, 16) &&
+                 aligned_to(t.param, d.p_bf16 ? 8 : 16))
                   ? 1
                   : 0;
       chunks += (t.numel + muon::kAdamChunk - 1) / muon::kAdamChunk;

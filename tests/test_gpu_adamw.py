@@ -44,7 +44,8 @@ def run_case(sizes, dtype, steps, offset=0, seed=0):
         p0 = (0.02 * rng.standard_normal(n)).astype(np.float32)
         if dtype == "bf16":
             p0 = bf16_round(p0).astype(np.float32)
-        # a view starting `offset` elements into a buffer takes the scalar path
+        # a view starting `offset` elements into a buffer: 0 keeps the 32-byte alignment of
+        # the allocation (256-bit path), 4 leaves 16 bytes (128-bit path), 1 none (scalar)
         buf = torch.zeros(n + offset, dtype=tdt, device="cuda")
         P.append(buf[offset:])
         P[-1].copy_(torch.from_numpy(p0).to(tdt))
@@ -101,6 +102,11 @@ def test_adamw_matches_oracle_over_three_steps(dtype):
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_adamw_unaligned_views_take_the_scalar_path(dtype):
     run_case([5, 4099, 70001], dtype, steps=2, offset=1, seed=1)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_adamw_16_byte_views_take_the_128_bit_path(dtype):
+    run_case([5, 4099, 70001], dtype, steps=2, offset=4, seed=3)
 
 
 def test_adamw_many_tensors_split_over_launches():
