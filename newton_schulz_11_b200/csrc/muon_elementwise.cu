@@ -7,6 +7,9 @@
 //                                          e' the exponent of hi raised to at least -113)
 //   partial[chunk] = sum of u^2            for ||u||_F of the listing's G.norm()
 //
+// Rows whose length is a multiple of 8 are read and written eight elements at a time
+// (256-bit accesses on 32-byte aligned rows, two 128-bit ones on 16-byte aligned rows,
+// the same element order either way); other rows four at a time, or one by one.
 // followed by a per-matrix finalisation s = 1 / (||u||_F + eps) in a fixed order
 // (deterministic: no atomics).  One CTA handles one chunk of whole rows of one
 // matrix; rows are read with 128-bit loads when the layout allows it.
@@ -61,7 +64,56 @@ __global__ void __launch_bounds__(kEwThreads) muon_momentum_kernel(const __grid_
   const int nesterov = p.nesterov, ns_only = p.ns_only;
   float acc = 0.f;
 
-  if (t.vec) {
+  if (t.vec >= 2) {
+    // eight elements per thread and iteration: one 256-bit access per row segment where
+    // the rows are 32-byte aligned (vec 2), two 128-bit ones where they are 16-byte
+    // aligned (vec 3); both visit the elements in the same order, so the sums of squares
+    // and everything after them do not depend on the alignment
+    const bool v8 = t.vec == 2;
+    const int c8 = t.cols >> 3;
+    const int total = (r1 - r0) * c8;
+    for (int idx = threadIdx.x; idx < total; idx += kEwThreads) {
+      const int rr = idx / c8;
+      const int c = (idx - rr * c8) << 3;
+      const int r = r0 + rr;
+      const float* gp = t.g + static_cast<int64_t>(r) * t.ld_g + c;
+      float* mp = t.m + static_cast<int64_t>(r) * t.ld_m + c;
+      float g[8], m[8], u[8];
+      if (v8) {
+        ld_global_cs_v8(gp, g);
+      } else {
+        const float4 g0 = __ldcs(reinterpret_cast<const float4*>(gp)), g1 = __ldcs(reinterpret_cast<const float4*>(gp) + 1);
+        g[0] = g0.x, g[1] = g0.y, g[2] = g0.z, g[3] = g0.w, g[4] = g1.x, g[5] = g1.y, g[6] = g1.z, g[7] = g1.w;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) m[j] = 0.f;
+      if (!ns_only) {
+        if (v8) {
+          ld_global_cs_v8(mp, m);
+        } else {
+          const float4 m0 = __ldcs(reinterpret_cast<const float4*>(mp)), m1 = __ldcs(reinterpret_cast<const float4*>(mp) + 1);
+          m[0] = m0.x, m[1] = m0.y, m[2] = m0.z, m[3] = m0.w, m[4] = m1.x, m[5] = m1.y, m[6] = m1.z, m[7] = m1.w;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) u[j] = ew_one(g[j], m[j], beta, nesterov, ns_only);
+      if (!ns_only) {
+        if (v8) {
+          st_global_cs_v8(mp, m);
+        } else {
+          __stcs(reinterpret_cast<float4*>(mp), make_float4(m[0], m[1], m[2], m[3]));
+          __stcs(reinterpret_cast<float4*>(mp) + 1, make_float4(m[4], m[5], m[6], m[7]));
+        }
+      }
+      uint32_t h01, h23, h45, h67, l0, l1;
+      split_hi_lo8x4(u[0], u[1], u[2], u[3], h01, h23, l0);
+      split_hi_lo8x4(u[4], u[5], u[6], u[7], h45, h67, l1);
+      *reinterpret_cast<uint4*>(t.hi + static_cast<int64_t>(r) * t.ldx + c) = make_uint4(h01, h23, h45, h67);
+      *reinterpret_cast<uint2*>(t.lo + static_cast<int64_t>(r) * t.ldl + c) = make_uint2(l0, l1);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc = fmaf(u[j], u[j], acc);
+    }
+  } else if (t.vec) {
     const int c4 = t.cols >> 2;
     const int total = (r1 - r0) * c4;
     for (int idx = threadIdx.x; idx < total; idx += kEwThreads) {

@@ -469,7 +469,12 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
       e.chunk_begin = w.chunk_begin[local];
       e.nchunks = w.nchunks[local];
       const bool mom_vec = t.momentum == nullptr || (aligned(t.momentum, 16) && t.ld_mom % 4 == 0);
-      e.vec = (t.cols % 4 == 0 && t.ld_grad % 4 == 0 && aligned(t.grad, 16) && mom_vec) ? 1 : 0;
+      const bool mom_v8 = t.momentum == nullptr || (aligned(t.momentum, 32) && t.ld_mom % 8 == 0);
+      const bool vec16 = t.ld_grad % 4 == 0 && aligned(t.grad, 16) && mom_vec;
+      const bool vec32 = t.ld_grad % 8 == 0 && aligned(t.grad, 32) && mom_v8;
+      // eight elements per thread when the rows allow it: 2 (32-byte rows), 3 (16-byte rows);
+      // else 1 (four elements, 16-byte rows) or 0 (one by one)
+      e.vec = (t.cols % 8 == 0 && vec32) ? 2 : (t.cols % 8 == 0 && vec16) ? 3 : (t.cols % 4 == 0 && vec16) ? 1 : 0;
 
       L->shape_scale[local] =
           t.shape_scale > 0.f ? t.shape_scale

@@ -107,7 +107,7 @@ struct EwMat {
   int32_t rows_per_chunk;
   int32_t chunk_begin;
   int32_t nchunks;
-  int32_t vec;            // float4 path allowed (cols, lds multiples of 4, 16-byte bases)
+  int32_t vec;            // 2: 8 per thread, 256-bit; 3: 8 per thread, 128-bit; 1: 4 per thread; 0: scalar
   int32_t pad_;
 };
 
