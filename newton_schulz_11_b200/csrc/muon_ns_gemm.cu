@@ -601,7 +601,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
     for (int q = 0; q < 4; ++q) mbar_init(&efull[q], 1);
     mbar_init(pdone, 1);
     *abort_flag = 0;
-    *epi_flag = 0;
+    *epi_flag = 1;  // live; an epilogue wait that gives up clears it
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -796,17 +796,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
       if constexpr (MODE == kApplyLast) wq_ok = load_w_segment<MODE, NCW>(p, cd, tl, rank, r, NCW * h, wq);
 #pragma unroll 1
       for (int q = 0; q < 4; ++q) {
-        // One warp waits (for the accumulator first, then for the inputs: kApply one
-        // quarter at a time, kApplyLast all four at once); the rest learn the outcome at
-        // the barrier, so every epilogue warp leaves together.
-        if (MODE == kApply || q == 0) {
+        // kApply: every warp waits for the accumulator (first quarter) and quarter q's
+        // inputs itself.  A warp whose wait gives up clears the live flag and skips the
+        // quarter's arithmetic but still meets the others at the "quarter q is final"
+        // barrier, after which all of them see the flag and leave together.
+        // kApplyLast: one warp waits (for the accumulator, then all four quarters); the
+        // rest learn the outcome at the barrier.
+        bool qok = true;
+        if constexpr (MODE == kApply) {
+          qok = q > 0 || warp_wait(&tfull[acc], aph, wd, kSiteEpilogueFull);
+          if (qok) qok = warp_wait(&efull[q], kpar, wd, kSiteEpilogueIn);
+          __syncwarp();  // lane 0's acquire of the landed data orders the other lanes' reads
+          if (lane == 0) {
+            if (!qok) *epi_flag = 0;
+            else if (ew == 0) pending &= ~(1u << q);
+          }
+        } else if (q == 0) {
           if (ew == 0) {
-            bool ok = q > 0 || warp_wait(&tfull[acc], aph, wd, kSiteEpilogueFull);
-            const int q_hi = MODE == kApply ? q : 3;
-            for (int qq = q; ok && qq <= q_hi; ++qq) ok = warp_wait(&efull[qq], kpar, wd, kSiteEpilogueIn);
+            bool ok = warp_wait(&tfull[acc], aph, wd, kSiteEpilogueFull);
+            for (int qq = 0; ok && qq < 4; ++qq) ok = warp_wait(&efull[qq], kpar, wd, kSiteEpilogueIn);
             if (lane == 0) {
               *epi_flag = ok ? 1 : 0;
-              if (ok) pending &= ~(((2u << q_hi) - 1u) & ~((1u << q) - 1u));
+              if (ok) pending &= ~0xFu;
             }
           }
           named_barrier(1, NT);
@@ -841,7 +852,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
 #pragma unroll
           for (int i = 0; i < NCW / 8; ++i) wq[i] = wn[i];
           wq_ok = wn_ok;
-        } else {
+        } else if (qok) {
           apply_staged<MODE, NCW>(p, cd, tl, rank, r, c0, tacc + c0, hib, lob, sc);
         }
         if (q == 3) {
@@ -851,7 +862,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
         }
         if constexpr (MODE == kApply) {
           fence_proxy_async_smem();
-          named_barrier(1, NT);  // quarter q is final
+          named_barrier(1, NT);  // quarter q is final (or some warp's wait gave up)
+          if (*epi_flag == 0) {
+            live = false;
+            break;
+          }
           if (leader) {
             store_region(&p.map_out[tl.cls], hib, q, 1, row0, col0, tl.mat);
             tma_store_3d(&p.map_out2[tl.cls], lob + q * kLoBlock, col0 + 64 * q, row0, tl.mat);
