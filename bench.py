@@ -38,11 +38,11 @@ KINDS = ("momentum", "norm", "gram", "poly", "apply", "apply_last")
 # the benchmarked workload, keyed by kernel kind; valid only while the kernel sources hash to
 # `source_hash` (kernel_source_hash: comments and layout do not count; see profiles/).
 # Filled in from the committed ncu summary.
-NCU_TRAFFIC = {"source_hash": "aa0655206805728c", "workload": DEFAULT_WORKLOAD,
-               "bytes_per_launch": {"momentum": 1222763776, "norm": 29696, "gram": 209649305,
-                                    "poly": 125845555, "apply": 547166528, "apply_last": 658015232}}
+NCU_TRAFFIC = {"source_hash": "1bbc922b404858ed", "workload": DEFAULT_WORKLOAD,
+               "bytes_per_launch": {"momentum": 1221587712, "norm": 29952, "gram": 210905241,
+                                    "poly": 125945241, "apply": 548369472, "apply_last": 658044416}}
 # the same for the AdamW path (workload gpt2-124m-adamw-params, one launch per step)
-NCU_TRAFFIC_ADAMW = {"source_hash": "aa0655206805728c", "bytes_per_launch": 893828608}
+NCU_TRAFFIC_ADAMW = {"source_hash": "1bbc922b404858ed", "bytes_per_launch": 894222080}
 
 
 def _code_only(text: str) -> str:
