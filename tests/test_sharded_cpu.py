@@ -148,3 +148,26 @@ def test_sharded_step_matches_single_process(tmp_path, world, reduce_grads, wave
         mine = [[i for i in range(len(SHAPES)) if owners[i] == r and res[r]["waves"][i] == j]
                 for j in range(max(res[r]["waves"]) + 1)]
         assert res[r]["calls"] == [c for c in mine if c] * 2
+
+
+def test_flat_buffers_keep_views_aligned_and_disjoint():
+    sys.path.insert(0, ROOT)
+    from newton_schulz_11_b200.distributed import _PAD, _Flat
+
+    shapes = [(3, 5), (8, 8), (1, 1), (16, 24)]
+    for dtype in (torch.float32, torch.bfloat16):
+        f = _Flat(shapes, dtype, torch.device("cpu"))
+        base = f.buf.data_ptr()
+        spans = []
+        for v, (r, c) in zip(f.views, shapes):
+            assert tuple(v.shape) == (r, c) and v.is_contiguous()
+            off = (v.data_ptr() - base) // f.buf.element_size()
+            assert off % _PAD == 0
+            spans.append((off, off + r * c))
+        spans.sort()
+        assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))
+        src = [torch.randn(s).to(dtype) for s in shapes]
+        f.pack(src)
+        dst = [torch.empty(s, dtype=dtype) for s in shapes]
+        f.unpack(dst)
+        assert all(torch.equal(a, b) for a, b in zip(src, dst))
