@@ -9,7 +9,6 @@ from .muon_oracle import (  # noqa: F401
     gram,
     momentum_update,
     muon_step,
-    muon_step_group,
     nesterov_input,
     newton_schulz,
     parameter_update,

@@ -41,7 +41,7 @@ invariances and tiny hand-checkable inputs.
 from __future__ import annotations
 
 import math
-from typing import Iterable, List, Optional, Sequence, Tuple
+from typing import Optional, Sequence, Tuple
 
 import numpy as np
 
@@ -139,8 +139,3 @@ def muon_step(W: np.ndarray, g: np.ndarray, m: np.ndarray, *, lr: float, beta: f
     W_new = parameter_update(W, O, lr, weight_decay, scale)
     return W_new, m_new, O
 
-
-def muon_step_group(Ws: Iterable[np.ndarray], gs: Iterable[np.ndarray], ms: Iterable[np.ndarray],
-                    **kw) -> List[Tuple[np.ndarray, np.ndarray, np.ndarray]]:
-    """The grouped call: every matrix is an independent problem, taken one after another."""
-    return [muon_step(W, g, m, **kw) for W, g, m in zip(Ws, gs, ms)]
