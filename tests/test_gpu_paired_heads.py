@@ -11,7 +11,7 @@ import pytest
 
 import oracle
 from newton_schulz_11_b200 import inputs
-from tests.gpu_util import rel_fro, require_gpu, to_np, torch
+from tests.gpu_util import bf16_ulp, rel_fro, require_gpu, to_np, torch
 
 pytestmark = pytest.mark.gpu
 QUINTIC5 = [oracle.QUINTIC] * 5
@@ -52,8 +52,16 @@ def test_head_blocks_match_the_oracle_per_block(heads_per_block):
             g = to_np(G[i])[sl].astype(np.float64)
             _, m_ref, O_ref = oracle.muon_step(W_in[i][sl].astype(np.float64), g, M_in[i][sl].astype(np.float64),
                                                lr=0.02, beta=0.95, weight_decay=0.01, nesterov=True, coeffs=QUINTIC5)
-            assert rel_fro(to_np(outs[k]), O_ref) <= 2e-2, (i, j)
+            O_gpu = to_np(outs[k])
+            assert rel_fro(O_gpu, O_ref) <= 2e-2, (i, j)
             assert rel_fro(to_np(M[i])[sl], m_ref) <= 1e-6, (i, j)
+            # W of the block: within one bf16 ulp of the oracle's update of the GPU's own O,
+            # plus the fp32 evaluation error (see check_bf16_update in the parity tests)
+            r, c = O_gpu.shape
+            scale = oracle.default_shape_scale(r, c)
+            W_exp = oracle.parameter_update(W_in[i][sl].astype(np.float64), O_gpu, 0.02, 0.01, scale)
+            bound = bf16_ulp(W_exp) + 2.0 ** -23 * (np.abs(W_in[i][sl]) + 0.02 * scale * np.abs(O_gpu))
+            assert (np.abs(to_np(W[i].float())[sl] - W_exp) <= bound).all(), (i, j)
             k += 1
 
 
