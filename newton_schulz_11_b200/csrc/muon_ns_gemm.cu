@@ -30,7 +30,8 @@
 // and  Y <- a Y + Y B  (B symmetric), so operand majorness is a per-class run-time
 // property of the launch.
 //
-// Roles in each CTA (320 threads, one CTA per SM, persistent over a flat tile list):
+// Roles in each CTA (320 threads, 352 in the staged applies; one CTA per SM, persistent
+// over a flat tile list):
 //   warp 0      one thread: TMA loads of 64 x 64 bf16 boxes (128-byte swizzle) into a
 //               ring of shared-memory stages
 //   warp 1      allocates TMEM for the pair (two fp32 accumulators of 128 x 256); in
@@ -38,7 +39,11 @@
 //   warps 2..9  epilogue: tcgen05.ld (TMEM lane = tile row; warps w and w + 4 share a
 //               lane quarter and split the columns), fused coefficient math in fp32,
 //               results staged in shared memory (128-byte swizzle) and written by TMA
-//               stores, one 128 x 128 block at a time.
+//               stores, one 128 x 128 block at a time (the staged applies write theirs
+//               straight from registers instead)
+//   warp 10     staged applies only: TMA loads of the epilogue's inputs (the tile's old hi
+//               and lo), a 64-column quarter at a time, each as soon as every epilogue warp
+//               has read the quarter it replaces
 // The epilogue of tile t overlaps the main loop of tile t + 1.
 #include "muon_device.cuh"
 #include "muon_params.h"
@@ -56,14 +61,17 @@ namespace muon {
 //     Gram        five stages; two 32 KB output staging buffers (stores of one quarter
 //                 drain while the next is written)
 //     polynomial  three stages; two output buffers; the tile's A block (64 KB) staged
-//     apply       four stages; the tile's hi (64 KB) and 8-bit lo (32 KB) staged and
-//                 updated in place
-template <int MODE, bool SMALL = false>
+//     apply       four stages; the tile's old hi (64 KB) and 8-bit lo (32 KB) staged by the
+//                 loader warp; the new hi and lo (or W and O) written with 32-byte global
+//                 stores, so no epilogue warp waits for a store or for another warp
+template <int MODE, int VAR = kStreamed>
 struct Lay {
   static constexpr bool kSym = MODE == kGram || MODE == kPoly;
+  static constexpr bool SMALL = VAR == kStaged;
+  static constexpr bool kLoader = SMALL && !kSym;  // staged applies: a warp stages the epilogue's inputs
   static constexpr int TM = 256;  // pair tile rows (128 per CTA)
   static constexpr int TN = 256;  // pair tile columns = UMMA N
-  static constexpr int BK = SMALL ? 64 : 128;
+  static constexpr int BK = VAR == kStreamed ? 128 : 64;
   static constexpr int S = !SMALL ? 3 : (MODE == kGram ? 5 : (kSym ? 3 : 4));
   // epilogue warps (16 for the staged apply measured no faster than 8)
   static constexpr int NEPI = 8;
@@ -79,7 +87,8 @@ struct Lay {
   static constexpr int kBarOff = kRing + kEpi;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;
   static constexpr int kEpiThreads = 32 * NEPI;
-  static constexpr int kThreads = 64 + kEpiThreads;
+  static constexpr int kLoaderWarp = 2 + NEPI;
+  static constexpr int kThreads = 64 + kEpiThreads + (kLoader ? 32 : 0);
   static constexpr int kTmemCols = 2 * TN;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
@@ -276,6 +285,41 @@ __device__ __forceinline__ void load_row32_u8(const uint8_t* row, int valid, boo
       if (k <= 0) e[j] = kZero4;
       else if (k < 4) e[j] = (e[j] & ((1u << (8 * k)) - 1u)) | (kZero4 & ~((1u << (8 * k)) - 1u));
     }
+  }
+}
+
+// 32 consecutive bf16 of one row (16 words, element 2i in the low half of word i) to `row`,
+// the first `valid` of them only; v8: the segment is 32-byte aligned.
+__device__ __forceinline__ void store_hi32(__nv_bfloat16* row, int valid, bool v8, const uint32_t (&w)[16]) {
+  if (valid >= 32) {
+    if (v8) {
+      st_global_v8(row, make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]));
+      st_global_v8(row + 16, make_uint4(w[8], w[9], w[10], w[11]), make_uint4(w[12], w[13], w[14], w[15]));
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        reinterpret_cast<uint4*>(row)[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < valid) put_bf16(row + j, (j & 1) ? (w[j >> 1] >> 16) : (w[j >> 1] & 0xFFFFu));
+  }
+}
+
+// 32 stored residual bytes (8 words, element j in byte j % 4 of word j / 4), the first `valid`.
+__device__ __forceinline__ void store_lo32(uint8_t* row, int valid, bool v8, const uint32_t (&w)[8]) {
+  if (valid >= 32) {
+    if (v8) {
+      st_global_v8(row, make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]));
+    } else {
+      reinterpret_cast<uint4*>(row)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      reinterpret_cast<uint4*>(row)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < valid) row[j] = static_cast<uint8_t>(w[j >> 2] >> (8 * (j & 3)));
   }
 }
 
@@ -483,7 +527,7 @@ template <int MODE>
 __device__ __forceinline__ void apply_quarter(const typename ParamsOf<MODE>::type& p, const ClassDesc& cd,
                                               const Tile& tl, int rank, int r, int c0, uint32_t tcol,
                                               const uint4 (&xh4)[4], const uint4 (&xl4)[2], float s,
-                                              uint32_t (&hb)[16], uint32_t (&lb)[8]) {
+                                              uint32_t (&hb)[16], uint32_t (&lb)[8], const uint4* w_pre = nullptr) {
   uint32_t v[32];
   tmem_ld_32x32b_x32(tcol, v);
   float x[32];
@@ -498,7 +542,7 @@ __device__ __forceinline__ void apply_quarter(const typename ParamsOf<MODE>::typ
   } else {
     (void)hb;
     (void)lb;
-    write_update<MODE>(p, cd, tl, rank, r, c0, x);
+    write_update<MODE>(p, cd, tl, rank, r, c0, x, w_pre);
   }
 }
 
@@ -510,58 +554,13 @@ __device__ __forceinline__ void tmem_ld_row(uint32_t taddr, uint32_t (&v)[NC]) {
     tmem_ld_32x32b_x16(taddr, v);
 }
 
-// Staged variant of the same update for NC (16 or 32) columns: the old pair is read from
-// the staged region (hi at hib in the 128-byte swizzle, lo at lob in 64-byte-swizzled 8 KB
-// quarter blocks); kApply writes the new pair back in place (the region is then stored by
-// TMA), kApplyLast updates W and/or writes O (w_pre: this thread's W segment, loaded
-// ahead, or nullptr).
-template <int MODE, int NC>
-__device__ __forceinline__ void apply_staged(const typename ParamsOf<MODE>::type& p, const ClassDesc& cd,
-                                             const Tile& tl, int rank, int r, int c0, uint32_t tcol, uint8_t* hib,
-                                             uint8_t* lob, float s, const uint4* w_pre = nullptr) {
-  uint32_t v[NC];
-  tmem_ld_row<NC>(tcol, v);
-  uint4 xh4[NC / 8], xl4[NC / 16];
-#pragma unroll
-  for (int q = 0; q < NC / 8; ++q) xh4[q] = *reinterpret_cast<const uint4*>(hib + region_chunk(r, (c0 >> 3) + q));
-  // quarter c0 / 64 of the lo block; this thread's bytes are chunks lc .. of its row
-  uint8_t* lq = lob + ((c0 >> 6) << 13);
-  const int lc = (c0 & 63) >> 4;
-#pragma unroll
-  for (int q = 0; q < NC / 16; ++q) xl4[q] = *reinterpret_cast<const uint4*>(lq + lo8_chunk(r, lc + q));
-  float x[NC];
-  decode_row<NC>(reinterpret_cast<const uint32_t*>(xh4), reinterpret_cast<const uint32_t*>(xl4), x);
-  tmem_wait_ld();
-#pragma unroll
-  for (int j = 0; j < NC; ++j) x[j] = fmaf(p.a, x[j], __uint_as_float(v[j]));
-  if (s != 1.f) {  // iteration 0 only (uniform)
-#pragma unroll
-    for (int j = 0; j < NC; ++j) x[j] *= s;
-  }
-  if constexpr (MODE == kApply) {
-    uint32_t hb[NC / 2], lb[NC / 4];
-#pragma unroll
-    for (int k = 0; k < NC / 4; ++k)
-      split_hi_lo8x4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3], hb[2 * k], hb[2 * k + 1], lb[k]);
-#pragma unroll
-    for (int q = 0; q < NC / 8; ++q)
-      *reinterpret_cast<uint4*>(hib + region_chunk(r, (c0 >> 3) + q)) =
-          make_uint4(hb[4 * q], hb[4 * q + 1], hb[4 * q + 2], hb[4 * q + 3]);
-#pragma unroll
-    for (int q = 0; q < NC / 16; ++q)
-      *reinterpret_cast<uint4*>(lq + lo8_chunk(r, lc + q)) = make_uint4(lb[4 * q], lb[4 * q + 1], lb[4 * q + 2],
-                                                                        lb[4 * q + 3]);
-  } else {
-    write_update<MODE, NC>(p, cd, tl, rank, r, c0, x, w_pre);
-  }
-}
-
 // ------------------------------------------------------------------ the kernel
 
-template <int MODE, bool SMALL>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kThreads, 1)
+template <int MODE, int VAR>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, VAR>::kThreads, 1)
     muon_ns_gemm_kernel(const __grid_constant__ typename ParamsOf<MODE>::type p) {
-  using L = Lay<MODE, SMALL>;
+  using L = Lay<MODE, VAR>;
+  constexpr bool SMALL = L::SMALL;
   constexpr int S = L::S;
   constexpr bool kSym = L::kSym;
   constexpr int NT = L::kEpiThreads;
@@ -575,7 +574,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
   uint64_t* tdown = tempty + 2;
   uint64_t* efull = tdown + 1;  // staged variant: quarter q of the tile's hi/lo inputs has landed
   uint64_t* pdone = efull + 4;  // used in the leader CTA: the peer's producer has finished
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pdone + 1);
+  uint64_t* consumed = pdone + 1;  // staged apply: every epilogue warp has read quarter q
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(consumed + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* epi_flag = abort_flag + 1;
   volatile uint32_t* peer_issued = reinterpret_cast<volatile uint32_t*>(epi_flag + 1);  // leader CTA
@@ -600,6 +600,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
     mbar_init(tdown, 1);
     for (int q = 0; q < 4; ++q) mbar_init(&efull[q], 1);
     mbar_init(pdone, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(&consumed[q], L::NEPI);
     *abort_flag = 0;
     *epi_flag = 1;  // live; an epilogue wait that gives up clears it
     fence_mbar_init();
@@ -608,7 +609,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
     for (int c = 0; c < p.num_classes; ++c) {
       tma_prefetch_desc(&p.map_a[c]);
       tma_prefetch_desc(&p.map_b[c]);
-      if (SMALL) {
+      if (VAR != kStreamed) {
         tma_prefetch_desc(&p.map_in[c]);
         tma_prefetch_desc(&p.map_out2[c]);
       }
@@ -747,159 +748,140 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
       }
       quiet_wait(tdown, 0, tb);
     }
+  } else if (L::kLoader && warp == L::kLoaderWarp) {
+    // ---------------------------------------------------------------- epilogue input loader (both CTAs)
+    // Quarter q of tile k's old hi and lo (this CTA's 128 rows x 64 columns) is loaded into
+    // its staging slot once every epilogue warp has read quarter q of tile k - 1.
+    if (lane == 0) {
+      uint8_t* hib = epi;
+      uint8_t* lob = epi + 4 * L::kHalf;
+      int k = 0;
+      bool ok = true;
+      uint32_t issued = 0, last_par = 0;  // per quarter: a load issued; the parity of the last one
+      for (int t = pair; ok && t < p.total_tiles; t += npairs, ++k) {
+        const Tile tl = decode_tile<MODE>(p, t);
+        const int row0 = L::TM * tl.I + kBM * rank, col0 = L::TN * tl.J;
+        for (int q = 0; q < 4; ++q) {
+          if (k > 0 && !mbar_wait(&consumed[q], static_cast<uint32_t>(k - 1) & 1u, wd, kSiteProducerEpi)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&efull[q], L::kHalf + kLoBlock);
+          load_region_quarter(hib, &p.map_in[tl.cls], &efull[q], q, row0, col0, tl.mat);
+          tma_load_3d(lob + q * kLoBlock, &p.map_out2[tl.cls], &efull[q], col0 + 64 * q, row0, tl.mat);
+          issued |= 1u << q;
+          last_par = (last_par & ~(1u << q)) | ((static_cast<uint32_t>(k) & 1u) << q);
+        }
+      }
+      // Before the CTA leaves, every load issued has landed.  A quarter has at most one load
+      // outstanding: the one before it was waited for by every epilogue warp.
+      for (int q = 0; q < 4; ++q)
+        if (issued & (1u << q)) quiet_wait(&efull[q], (last_par >> q) & 1u, tb);
+    }
   } else if constexpr (SMALL && !kSym) {
     // ---------------------------------------------------------------- staged apply epilogue (both CTAs)
-    // The tile's old hi/lo (128 x 256 each per CTA) live in the staging region as four
-    // 64-column quarters, each with its own barrier.  Quarter q is updated (kApply: in
-    // place, then stored by TMA) and, as soon as nothing reads it any more, refilled with
-    // quarter q of this pair's next tile, so the loads run three quarters ahead of use.
+    // The tile's old hi and lo (128 x 256 each per CTA) arrive in shared memory as four
+    // 64-column quarters from the loader warp.  Each warp waits for the accumulator and each
+    // quarter itself, reads its part, tells the loader it is done with the quarter, and
+    // writes its results straight to global memory: the new pair (kApply) or W and/or O
+    // (kApplyLast).  The epilogue warps never wait for one another.
     const int ew = warp - 2;
     const int q4 = warp & 3;  // TMEM lanes 32 q4 .. 32 q4 + 31 belong to this warp
-    constexpr int NCW = 256 / L::NEPI;  // columns of each quarter per thread (16 with 16 warps)
-    const int h = ew >> 2;              // which NCW columns of each quarter
+    const int h = ew >> 2;    // which 32 columns of each 64-column quarter
     const int r = q4 * 32 + lane;
-    const bool leader = threadIdx.x == 64;  // also the thread that waits on the barriers
     const uint32_t tempty0 = map_to_rank(smem_u32(tempty), 0);
     uint8_t* hib = epi;
-    uint8_t* lob = epi + 4 * L::kHalf;  // four 8 KB blocks of 8-bit lo, one per quarter
+    uint8_t* lob = epi + 4 * L::kHalf;
     int acc = 0;
     uint32_t aph = 0;
-    uint32_t pending = 0, pend_par = 0;  // leader: quarter loads not yet waited for, and their parity
-    auto load_quarter = [&](const Tile& nx, int q, uint32_t par) {
-      const int row0 = L::TM * nx.I + kBM * rank, col0 = L::TN * nx.J;
-      mbar_arrive_expect_tx(&efull[q], L::kHalf + kLoBlock);
-      load_region_quarter(hib, &p.map_in[nx.cls], &efull[q], q, row0, col0, nx.mat);
-      tma_load_3d(lob + q * kLoBlock, &p.map_out2[nx.cls], &efull[q], col0 + 64 * q, row0, nx.mat);
-      pending |= 1u << q;
-      pend_par = (pend_par & ~(1u << q)) | (par << q);
-    };
-    if (leader && pair < p.total_tiles) {
-      const Tile first = decode_tile<MODE>(p, pair);
-      for (int q = 0; q < 4; ++q) load_quarter(first, q, 0u);
-    }
     int k = 0;
-    bool live = true;
-    for (int t = pair; live && t < p.total_tiles; t += npairs, ++k) {
+    for (int t = pair; t < p.total_tiles; t += npairs, ++k) {
       const Tile tl = decode_tile<MODE>(p, t);
       const ClassDesc& cd = p.cls[tl.cls];
       const uint32_t kpar = static_cast<uint32_t>(k) & 1u;
-      const bool has_next = t + npairs < p.total_tiles;
-      Tile nx = tl;
-      if (has_next) nx = decode_tile<MODE>(p, t + npairs);
+      const int Rx = L::TM * tl.I + kBM * rank + r;
+      const bool live = Rx < cd.rows;
+      const bool hv8 = (cd.ldx & 15) == 0, lv8 = (cd.ldl & 31) == 0;  // 32-byte rows
+      const int64_t xoff = tl.mat * cd.x_stride + static_cast<int64_t>(Rx) * cd.ldx;
+      const int64_t loff = tl.mat * cd.lo_stride + static_cast<int64_t>(Rx) * cd.ldl;
       const float sc = p.first_iter ? p.scale[cd.mat_base + tl.mat] : 1.f;
-      const int row0 = L::TM * tl.I + kBM * rank, col0 = L::TN * tl.J;
       const uint32_t tacc = tmem_base + static_cast<uint32_t>(acc * L::TN) + (static_cast<uint32_t>(q4 * 32) << 16);
-      // kApplyLast: this thread's bf16 W segment for the quarter after the one being
-      // computed is loaded one quarter ahead (the first before the accumulator wait)
-      uint4 wq[NCW / 8];
+      uint4 wq[4];
       bool wq_ok = false;
-      if constexpr (MODE == kApplyLast) wq_ok = load_w_segment<MODE, NCW>(p, cd, tl, rank, r, NCW * h, wq);
+      if constexpr (MODE == kApplyLast) {
+        wq_ok = load_w_segment<MODE, 32>(p, cd, tl, rank, r, 32 * h, wq);
+        if (h == 0 && t + npairs < p.total_tiles) {  // warm L2 with this thread's row of W in the next tile
+          const Tile nx = decode_tile<MODE>(p, t + npairs);
+          const ClassDesc& nd = p.cls[nx.cls];
+          const UpdMat& un = p.upd[nd.mat_base + nx.mat];
+          const int Rn = L::TM * nx.I + kBM * rank + r, Cn = L::TN * nx.J;
+          if (un.param != nullptr && Rn < nd.rows) {
+            const int esz = un.param_bf16 ? 2 : 4;
+            const int bytes = (nd.cols - Cn < L::TN ? nd.cols - Cn : L::TN) * esz;
+            const char* row = static_cast<const char*>(un.param) + (static_cast<int64_t>(Rn) * un.ld_param + Cn) * esz;
+            for (int off = 0; off < bytes; off += 128) prefetch_l2(row + off);
+            prefetch_l2(row + bytes - 1);
+          }
+        }
+      }
+      bool ok = warp_wait(&tfull[acc], aph, wd, kSiteEpilogueFull);
+      if (ok) tc_fence_after();
 #pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
-        // kApply: every warp waits for the accumulator (first quarter) and quarter q's
-        // inputs itself.  A warp whose wait gives up clears the live flag and skips the
-        // quarter's arithmetic but still meets the others at the "quarter q is final"
-        // barrier, after which all of them see the flag and leave together.
-        // kApplyLast: one warp waits (for the accumulator, then all four quarters); the
-        // rest learn the outcome at the barrier.
-        bool qok = true;
-        if constexpr (MODE == kApply) {
-          qok = q > 0 || warp_wait(&tfull[acc], aph, wd, kSiteEpilogueFull);
-          if (qok) qok = warp_wait(&efull[q], kpar, wd, kSiteEpilogueIn);
-          __syncwarp();  // lane 0's acquire of the landed data orders the other lanes' reads
-          if (lane == 0) {
-            if (!qok) *epi_flag = 0;
-            else if (ew == 0) pending &= ~(1u << q);
-          }
-        } else if (q == 0) {
-          if (ew == 0) {
-            bool ok = warp_wait(&tfull[acc], aph, wd, kSiteEpilogueFull);
-            for (int qq = 0; ok && qq < 4; ++qq) ok = warp_wait(&efull[qq], kpar, wd, kSiteEpilogueIn);
-            if (lane == 0) {
-              *epi_flag = ok ? 1 : 0;
-              if (ok) pending &= ~0xFu;
-            }
-          }
-          named_barrier(1, NT);
-          if (*epi_flag == 0) {
-            live = false;
-            break;
-          }
-        }
-        if (q == 0) {
-          tc_fence_after();
-          if constexpr (MODE == kApplyLast) {
-            // warm L2 with this thread's row of W in the next tile
-            if (has_next) {
-              const ClassDesc& nd = p.cls[nx.cls];
-              const UpdMat& un = p.upd[nd.mat_base + nx.mat];
-              const int Rn = L::TM * nx.I + kBM * rank + r, Cn = L::TN * nx.J;
-              if (un.param != nullptr && Rn < nd.rows) {
-                const int esz = un.param_bf16 ? 2 : 4;
-                const int bytes = (nd.cols - Cn < L::TN ? nd.cols - Cn : L::TN) * esz;
-                const char* row = static_cast<const char*>(un.param) + (static_cast<int64_t>(Rn) * un.ld_param + Cn) * esz;
-                for (int off = 0; off < bytes; off += 128) prefetch_l2(row + off);
-                prefetch_l2(row + bytes - 1);
-              }
-            }
-          }
-        }
-        const int c0 = 64 * q + NCW * h;
-        if constexpr (MODE == kApplyLast) {
-          uint4 wn[NCW / 8];
-          const bool wn_ok = q < 3 && load_w_segment<MODE, NCW>(p, cd, tl, rank, r, c0 + 64, wn);
-          apply_staged<MODE, NCW>(p, cd, tl, rank, r, c0, tacc + c0, hib, lob, sc, wq_ok ? wq : nullptr);
+      for (int q = 0; ok && q < 4; ++q) {
+        ok = warp_wait(&efull[q], kpar, wd, kSiteEpilogueIn);
+        if (!ok) break;
+        const int c0 = 64 * q + 32 * h;
+        uint4 wn[4];
+        bool wn_ok = false;
+        if constexpr (MODE == kApplyLast) wn_ok = q < 3 && load_w_segment<MODE, 32>(p, cd, tl, rank, r, c0 + 64, wn);
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tacc + c0, v);
+        uint4 xh4[4], xl4[2];
 #pragma unroll
-          for (int i = 0; i < NCW / 8; ++i) wq[i] = wn[i];
-          wq_ok = wn_ok;
-        } else if (qok) {
-          apply_staged<MODE, NCW>(p, cd, tl, rank, r, c0, tacc + c0, hib, lob, sc);
-        }
+        for (int i = 0; i < 4; ++i) xh4[i] = *reinterpret_cast<const uint4*>(hib + region_chunk(r, (c0 >> 3) + i));
+        const uint8_t* lq = lob + (q << 13);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) xl4[i] = *reinterpret_cast<const uint4*>(lq + lo8_chunk(r, 2 * h + i));
+        float x[32];
+        decode_row<32>(reinterpret_cast<const uint32_t*>(xh4), reinterpret_cast<const uint32_t*>(xl4), x);
+        tmem_wait_ld();  // before any other asm: v is written asynchronously until here
+        // The slot may be refilled once every warp's reads of it have completed: the decode
+        // above consumed the loaded values, and the proxy fence orders these generic-proxy
+        // reads before the loader's TMA (async-proxy) write of the next tile's quarter.
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&consumed[q]);  // this warp is done with quarter q
         if (q == 3) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * static_cast<uint32_t>(acc));
         }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = fmaf(p.a, x[j], __uint_as_float(v[j]));
+        if (sc != 1.f) {  // iteration 0 only (uniform)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) x[j] *= sc;
+        }
         if constexpr (MODE == kApply) {
-          fence_proxy_async_smem();
-          named_barrier(1, NT);  // quarter q is final (or some warp's wait gave up)
-          if (*epi_flag == 0) {
-            live = false;
-            break;
-          }
-          if (leader) {
-            store_region(&p.map_out[tl.cls], hib, q, 1, row0, col0, tl.mat);
-            tma_store_3d(&p.map_out2[tl.cls], lob + q * kLoBlock, col0 + 64 * q, row0, tl.mat);
-            bulk_commit();
-            // the stores of quarter q - 1 have read their boxes: refill them
-            if (q > 0) {
-              bulk_wait_read<1>();
-              if (has_next) load_quarter(nx, q - 1, kpar ^ 1u);
-            }
-          }
+          uint32_t hb[16], lb[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            split_hi_lo8x4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3], hb[2 * i], hb[2 * i + 1], lb[i]);
+          const int C = L::TN * tl.J + c0;
+          store_hi32(cd.x_hi_next + xoff + C, live ? cd.cols - C : 0, hv8, hb);
+          store_lo32(cd.x_lo + loff + C, live ? cd.cols - C : 0, lv8, lb);
+        } else {
+          write_update<MODE, 32>(p, cd, tl, rank, r, c0, x, wq_ok ? wq : nullptr);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) wq[i] = wn[i];
+          wq_ok = wn_ok;
         }
       }
-      if (!live) break;
-      if constexpr (MODE == kApply) {
-        if (leader) {
-          bulk_wait_read<0>();
-          if (has_next) load_quarter(nx, 3, kpar ^ 1u);
-        }
-      } else {
-        fence_proxy_async_smem();
-        named_barrier(1, NT);  // nothing reads the region any more
-        if (leader && has_next)
-          for (int q = 0; q < 4; ++q) load_quarter(nx, q, kpar ^ 1u);
-      }
+      if (!ok) break;
       if (++acc == 2) {
         acc = 0;
         aph ^= 1u;
       }
-    }
-    if (leader) {
-      bulk_wait_all();
-      for (int q = 0; q < 4; ++q)
-        if (pending & (1u << q)) quiet_wait(&efull[q], (pend_par >> q) & 1u, tb);
     }
   } else if constexpr (SMALL) {
     // ---------------------------------------------------------------- staged symmetric epilogue (both CTAs)
@@ -1155,10 +1137,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, SMALL>::kT
   }
 }
 
-template <int MODE, bool SMALL>
+template <int MODE, int VAR>
 static cudaError_t launch_one(const typename ParamsOf<MODE>::type& p, int max_pairs, cudaStream_t stream) {
-  using L = Lay<MODE, SMALL>;
-  auto* kernel = muon_ns_gemm_kernel<MODE, SMALL>;
+  using L = Lay<MODE, VAR>;
+  auto* kernel = muon_ns_gemm_kernel<MODE, VAR>;
   static thread_local int configured_device = -1;
   static thread_local int resident_pairs = 0;
   int dev = 0;
@@ -1199,16 +1181,18 @@ int gemm_tile_cols() { return 256; }
 cudaError_t launch_gemm(int mode, const GemmParams* p, int max_pairs, cudaStream_t stream) {
   switch (mode) {
     case kGram:
-      return p->staged ? launch_one<kGram, true>(*p, max_pairs, stream) : launch_one<kGram, false>(*p, max_pairs, stream);
+      return p->staged == kStaged ? launch_one<kGram, kStaged>(*p, max_pairs, stream)
+                                  : launch_one<kGram, kStreamed>(*p, max_pairs, stream);
     case kPoly:
-      return p->staged ? launch_one<kPoly, true>(*p, max_pairs, stream) : launch_one<kPoly, false>(*p, max_pairs, stream);
+      return p->staged == kStaged ? launch_one<kPoly, kStaged>(*p, max_pairs, stream)
+                                  : launch_one<kPoly, kStreamed>(*p, max_pairs, stream);
     case kApply:
-      return p->staged ? launch_one<kApply, true>(*p, max_pairs, stream)
-                       : launch_one<kApply, false>(*p, max_pairs, stream);
+      return p->staged == kStaged ? launch_one<kApply, kStaged>(*p, max_pairs, stream)
+                                  : launch_one<kApply, kStreamed>(*p, max_pairs, stream);
     case kApplyLast: {
       const FinalParams& f = *static_cast<const FinalParams*>(p);
-      return p->staged ? launch_one<kApplyLast, true>(f, max_pairs, stream)
-                       : launch_one<kApplyLast, false>(f, max_pairs, stream);
+      return p->staged == kStaged ? launch_one<kApplyLast, kStaged>(f, max_pairs, stream)
+                                  : launch_one<kApplyLast, kStreamed>(f, max_pairs, stream);
     }
     default: return cudaErrorInvalidValue;
   }

@@ -23,6 +23,14 @@ enum GemmMode : int {
   kApplyLast = 3,  // same, then W <- W decay - lr_scale X and/or O <- X
 };
 
+// Kernel variants (GemmParams::staged):
+//   kStreamed  128-deep k-blocks in three 64 KB stages; epilogue inputs read into registers,
+//              outputs staged in shared memory and written by TMA stores
+//   kStaged    64-deep k-blocks; the epilogue's inputs staged in shared memory by TMA.  The
+//              Gram and the polynomial store through shared memory by TMA; the applies
+//              write their results straight from registers
+enum GemmVariant : int { kStreamed = 0, kStaged = 1 };
+
 enum WaitSite : int {
   kSiteProducerEmpty = 1,
   kSiteMmaTmemEmpty = 2,
@@ -83,7 +91,8 @@ struct GemmParams {
   ClassDesc cls[kMaxClasses];
   int32_t num_classes;
   int32_t total_tiles;
-  int32_t staged;                   // apply: the staged variant (operand maps with 64 x 64 boxes)
+  int32_t staged;                   // GemmVariant of the launch (staged: 64-deep k-blocks,
+                                    // MN-major operand maps with 64 x 64 boxes)
   int32_t first_iter;               // iteration 0: s^2 on the Gram, s on the apply
   float a, b, c;                    // this iteration's coefficients
   float decay;                      // 1 - lr * weight_decay (final epilogue)
@@ -108,7 +117,7 @@ struct EwMat {
   int32_t chunk_begin;
   int32_t nchunks;
   int32_t vec;            // 2: 8 per thread, 256-bit; 3: 8 per thread, 128-bit; 1: 4 per thread; 0: scalar
-  int32_t pad_;
+  int32_t index;          // the matrix's index in the caller's descriptor array
 };
 
 struct EwParams {
@@ -122,6 +131,11 @@ struct EwParams {
   float* partials;        // one fp32 sum of squares per chunk
   float* scale;           // per matrix: 1 / (||u|| + eps)
   float* norm;            // per matrix: ||u||
+  int32_t* status;        // workspace header: [0] code, [1] where, [2..3] count of non-finite u (uint64)
 };
+
+// Device status codes written into the workspace header (muon_status_t values).
+constexpr int kStatusTimeout = 7;
+constexpr int kStatusNonfinite = 10;
 
 }  // namespace muon
