@@ -61,7 +61,7 @@
 extern "C" {
 #endif
 
-#define MUON_ABI_VERSION 3
+#define MUON_ABI_VERSION 4
 #define MUON_MAX_NS_STEPS 16
 
 typedef enum {
@@ -74,8 +74,11 @@ typedef enum {
   MUON_ERR_CUDA = 6,               /* a CUDA runtime call or launch failed */
   MUON_ERR_TIMEOUT = 7,            /* device status only: a bounded wait ran out */
   MUON_ERR_NO_DEVICE = 8,          /* current device is not an sm_100 GPU */
-  MUON_ERR_STATIC_SCRATCH_LIMIT = 9 /* muon_newton_schulz_static: a matrix needs more
+  MUON_ERR_STATIC_SCRATCH_LIMIT = 9, /* muon_newton_schulz_static: a matrix needs more
                                        scratch than MUON_STATIC_SCRATCH_BYTES */
+  MUON_ERR_NONFINITE = 10          /* device status only: a Newton-Schulz input u held a NaN
+                                      or an infinity (the values propagate into that
+                                      matrix's results; no other matrix is affected) */
 } muon_status_t;
 
 typedef enum { MUON_F32 = 0, MUON_BF16 = 1 } muon_dtype_t;
@@ -165,11 +168,25 @@ muon_status_t muon_scratch_view(const muon_matrix_t* mats, int n, int index,
                                 size_t workspace_bytes, muon_scratch_view_t* view);
 
 /*
- * Waits for `stream`, then reads the workspace's device status word into
- * *device_status (MUON_OK or MUON_ERR_TIMEOUT) and *where (the wait that gave up).
+ * Waits for `stream`, then reads the workspace's device status word into *device_status
+ * and *where (may be NULL):
+ *   MUON_OK
+ *   MUON_ERR_TIMEOUT    a bounded device-side wait ran out; *where = the wait site
+ *   MUON_ERR_NONFINITE  the elementwise pass found a NaN or an infinity in u (muon_step)
+ *                       or G (muon_newton_schulz); *where = the index, in that call's
+ *                       descriptor array, of a matrix that held one
+ * The first event recorded wins; the word is sticky until muon_workspace_init clears it.
+ * The pages define no status reporting (the step is a plain function there); the
+ * workspace argument replaces a per-stream query, since every call owns its workspace.
  */
 muon_status_t muon_device_status(const void* workspace, void* stream, int32_t* device_status,
                                  int32_t* where);
+
+/*
+ * Waits for `stream`, then reads how many non-finite values of u (or G) the elementwise
+ * passes that used this workspace have counted since muon_workspace_init cleared it.
+ */
+muon_status_t muon_nonfinite_count(const void* workspace, void* stream, int64_t* count);
 
 /*
  * Budget of every device-side wait, in microseconds (default 2,000,000 = 2 s).  A
@@ -246,8 +263,9 @@ muon_status_t muon_adamw_step(const muon_adamw_tensor_t* tensors, int n, float l
  *     fit in MUON_STATIC_SCRATCH_BYTES is rejected with MUON_ERR_STATIC_SCRATCH_LIMIT
  *     before anything is queued.  Sets that fit only together are processed in waves.
  *   - The first call on a device looks up the array's device address with the
- *     device current (cudaGetSymbolAddress).  Make that first call outside any
- *     stream capture.
+ *     device current (cudaGetSymbolAddress), and so does the first call after that
+ *     device's context has been re-created (e.g. by cudaDeviceReset).  Make those
+ *     calls outside any stream capture.
  *   - All calls share the one array, which keeps the last call's contents.  Each call
  *     clears the array's status word before its kernels run.  Calls whose kernels
  *     overlap on the GPU (other streams, other host threads) race on the array and

@@ -8,7 +8,7 @@ import threading
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libmuon_b200.so")
 
-MUON_ABI_VERSION = 3  # the version of include/muon_b200.h these bindings follow
+MUON_ABI_VERSION = 4  # the version of include/muon_b200.h these bindings follow
 MUON_OK = 0
 MUON_ERR_INVALID_ARG = 1
 MUON_ERR_ALIGNMENT = 2
@@ -19,6 +19,7 @@ MUON_ERR_CUDA = 6
 MUON_ERR_TIMEOUT = 7
 MUON_ERR_NO_DEVICE = 8
 MUON_ERR_STATIC_SCRATCH_LIMIT = 9
+MUON_ERR_NONFINITE = 10
 MUON_STATIC_SCRATCH_BYTES = 64 << 20
 
 MUON_F32 = 0
@@ -34,6 +35,7 @@ EXPORTS = (
     "muon_newton_schulz",
     "muon_scratch_view",
     "muon_device_status",
+    "muon_nonfinite_count",
     "muon_set_wait_timeout_us",
     "muon_profile_begin",
     "muon_profile_end",
@@ -142,6 +144,8 @@ def lib() -> ctypes.CDLL:
                                         P(MuonScratchView)]
         h.muon_device_status.restype = ctypes.c_int
         h.muon_device_status.argtypes = [ctypes.c_void_p, ctypes.c_void_p, P(ctypes.c_int32), P(ctypes.c_int32)]
+        h.muon_nonfinite_count.restype = ctypes.c_int
+        h.muon_nonfinite_count.argtypes = [ctypes.c_void_p, ctypes.c_void_p, P(ctypes.c_int64)]
         h.muon_set_wait_timeout_us.restype = ctypes.c_int
         h.muon_set_wait_timeout_us.argtypes = [ctypes.c_int64]
         h.muon_profile_begin.restype = ctypes.c_int

@@ -300,6 +300,13 @@ class PreparedMuonStep:
                                        ctypes.byref(where)), "muon_device_status")
         return int(code.value), int(where.value)
 
+    def nonfinite_count(self, stream=None) -> int:
+        """Non-finite values of u counted in this step's workspace since it was cleared."""
+        n = ctypes.c_int64(0)
+        check(lib().muon_nonfinite_count(self._ptr, _stream_handle(self.device, stream), ctypes.byref(n)),
+              "muon_nonfinite_count")
+        return int(n.value)
+
 
 class PreparedAdamW:
     """adamw_step for a fixed set of contiguous tensors: the descriptor array is built and
@@ -349,3 +356,17 @@ def device_status(workspace: Workspace, stream=None) -> Tuple[int, int]:
     check(lib().muon_device_status(workspace.buf.data_ptr(), s, ctypes.byref(code), ctypes.byref(where)),
           "muon_device_status")
     return int(code.value), int(where.value)
+
+
+def nonfinite_count(workspace: Workspace, stream=None) -> int:
+    """Non-finite values of u (or G) counted in `workspace` since it was last cleared."""
+    n = ctypes.c_int64(0)
+    check(lib().muon_nonfinite_count(workspace.buf.data_ptr(), _stream_handle(workspace.device, stream),
+                                     ctypes.byref(n)), "muon_nonfinite_count")
+    return int(n.value)
+
+
+def clear_device_status(workspace: Workspace, stream=None) -> None:
+    """Clears the status word and the non-finite count of `workspace` (queued on the stream)."""
+    check(lib().muon_workspace_init(workspace.buf.data_ptr(), workspace.buf.numel(),
+                                    _stream_handle(workspace.device, stream)), "muon_workspace_init")

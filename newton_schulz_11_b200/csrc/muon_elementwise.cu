@@ -6,6 +6,8 @@
 //                                          k + 64, k the residual in units of 2^(e' - 14),
 //                                          e' the exponent of hi raised to at least -113)
 //   partial[chunk] = sum of u^2            for ||u||_F of the listing's G.norm()
+//   non-finite u                           counted into the workspace header, which then
+//                                          reports MUON_ERR_NONFINITE (values propagate)
 //
 // Rows whose length is a multiple of 8 are read and written eight elements at a time
 // (256-bit accesses on 32-byte aligned rows, two 128-bit ones on 16-byte aligned rows,
@@ -63,6 +65,7 @@ __global__ void __launch_bounds__(kEwThreads) muon_momentum_kernel(const __grid_
   const float beta = p.beta;
   const int nesterov = p.nesterov, ns_only = p.ns_only;
   float acc = 0.f;
+  int nf = 0;  // non-finite values of u seen by this thread
 
   if (t.vec >= 2) {
     // eight elements per thread and iteration: one 256-bit access per row segment where
@@ -111,7 +114,10 @@ __global__ void __launch_bounds__(kEwThreads) muon_momentum_kernel(const __grid_
       *reinterpret_cast<uint4*>(t.hi + static_cast<int64_t>(r) * t.ldx + c) = make_uint4(h01, h23, h45, h67);
       *reinterpret_cast<uint2*>(t.lo + static_cast<int64_t>(r) * t.ldl + c) = make_uint2(l0, l1);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) acc = fmaf(u[j], u[j], acc);
+      for (int j = 0; j < 8; ++j) {
+        acc = fmaf(u[j], u[j], acc);
+        nf += isfinite(u[j]) ? 0 : 1;
+      }
     }
   } else if (t.vec) {
     const int c4 = t.cols >> 2;
@@ -137,6 +143,7 @@ __global__ void __launch_bounds__(kEwThreads) muon_momentum_kernel(const __grid_
       acc = fmaf(u1, u1, acc);
       acc = fmaf(u2, u2, acc);
       acc = fmaf(u3, u3, acc);
+      nf += (isfinite(u0) ? 0 : 1) + (isfinite(u1) ? 0 : 1) + (isfinite(u2) ? 0 : 1) + (isfinite(u3) ? 0 : 1);
     }
   } else {
     const int total = (r1 - r0) * t.cols;
@@ -153,10 +160,17 @@ __global__ void __launch_bounds__(kEwThreads) muon_momentum_kernel(const __grid_
       t.hi[static_cast<int64_t>(r) * t.ldx + c] = __ushort_as_bfloat16(static_cast<unsigned short>(h));
       t.lo[static_cast<int64_t>(r) * t.ldl + c] = static_cast<uint8_t>(lo8_encode(u, h));
       acc = fmaf(u, u, acc);
+      nf += isfinite(u) ? 0 : 1;
     }
   }
   const float s = block_sum(acc, red);
   if (threadIdx.x == 0) p.partials[chunk] = s;
+  if (__syncthreads_or(nf != 0)) {  // rare: this chunk holds a NaN or an infinity
+    const int w = __reduce_add_sync(0xffffffffu, nf);
+    if ((threadIdx.x & 31) == 0 && w != 0)
+      atomicAdd(reinterpret_cast<unsigned long long*>(p.status + 2), static_cast<unsigned long long>(w));
+    if (threadIdx.x == 0 && atomicCAS(&p.status[0], 0, kStatusNonfinite) == 0) atomicExch(&p.status[1], t.index);
+  }
 }
 
 // s_i = 1 / (sqrt(sum of the matrix's chunk partials) + eps), summed in fp64 in a

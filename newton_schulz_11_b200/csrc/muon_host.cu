@@ -41,7 +41,7 @@ constexpr size_t kHeaderBytes = 256;
 constexpr size_t kBufAlign = 1024;
 constexpr int64_t kChunkElems = 16384;
 constexpr int64_t kMaxSide = int64_t(1) << 24;
-constexpr int kStagedApplyMaxM = 1024;  // Gram side up to which the apply stages hi/lo by TMA
+constexpr int kStagedApplyMaxM = 1024;  // Gram side up to which the staged (64-deep) variants serve
 
 std::atomic<long long> g_timeout_us{2000000};
 
@@ -384,6 +384,7 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
   ew.partials = reinterpret_cast<float*>(ws + w.off_partials);
   ew.scale = scale;
   ew.norm = reinterpret_cast<float*>(ws + w.off_norm);
+  ew.status = status;
   L->shape_scale.resize(nw);
 
   int local = 0;
@@ -468,6 +469,7 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
       e.rows_per_chunk = w.rows_per_chunk[local];
       e.chunk_begin = w.chunk_begin[local];
       e.nchunks = w.nchunks[local];
+      e.index = gi;
       const bool mom_vec = t.momentum == nullptr || (aligned(t.momentum, 16) && t.ld_mom % 4 == 0);
       const bool mom_v8 = t.momentum == nullptr || (aligned(t.momentum, 32) && t.ld_mom % 8 == 0);
       const bool vec16 = t.ld_grad % 4 == 0 && aligned(t.grad, 16) && mom_vec;
@@ -524,8 +526,8 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
   for (int cur = 0; cur < 2; ++cur) {
     GemmParams g = base;
     GemmParams a = base;
-    g.staged = 0;
-    a.staged = staged ? 1 : 0;
+    g.staged = kStreamed;
+    a.staged = staged ? kStaged : kStreamed;
     for (int k = 0; k < nc; ++k) {
       const int ci = ord_sym[k];
       g.cls[k] = sym[ci];
@@ -560,7 +562,7 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
     static_cast<GemmParams&>(L->fin[cur]) = a;
   }
   GemmParams pp = base;
-  pp.staged = staged ? 1 : 0;
+  pp.staged = staged ? kStaged : kStreamed;
   for (int k = 0; k < nc; ++k) {
     const int ci = ord_app[k];  // the polynomial's reduction is m, like the apply's
     pp.cls[k] = sym[ci];
@@ -727,6 +729,7 @@ const char* muon_status_str(int status) {
     case MUON_ERR_TIMEOUT: return "device-side wait timed out";
     case MUON_ERR_NO_DEVICE: return "no sm_100 device is current";
     case MUON_ERR_STATIC_SCRATCH_LIMIT: return "a matrix needs more scratch than the static array holds (64 MiB)";
+    case MUON_ERR_NONFINITE: return "a Newton-Schulz input held NaN or infinite values";
     default: return "unknown status";
   }
 }
@@ -811,6 +814,16 @@ muon_status_t muon_device_status(const void* workspace, void* stream, int32_t* d
   return MUON_OK;
 }
 
+muon_status_t muon_nonfinite_count(const void* workspace, void* stream, int64_t* count) {
+  if (workspace == nullptr || count == nullptr) return MUON_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MUON_ERR_CUDA;
+  uint64_t c = 0;
+  if (cudaMemcpy(&c, static_cast<const uint8_t*>(workspace) + 8, sizeof(c), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MUON_ERR_CUDA;
+  *count = static_cast<int64_t>(c);
+  return MUON_OK;
+}
+
 muon_status_t muon_set_wait_timeout_us(int64_t us) {
   g_timeout_us.store(us > 0 ? us : 2000000);
   return MUON_OK;
@@ -860,19 +873,58 @@ constexpr int kMaxDevices = 64;
 // symbol; its device address comes from cudaGetSymbolAddress, per device.
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
+// The array's address on each device, with the id of the context it was looked up in.  A
+// context id is never reused within a process, so after the device's primary context has
+// been torn down and re-created (cudaDeviceReset), the first call looks the address up
+// again instead of using one from an unloaded module.
+struct StaticAddr {
+  unsigned long long ctx_id = 0;
+  void* addr = nullptr;
+};
 std::mutex g_static_mu;
-void* g_static_addr[kMaxDevices] = {};
+StaticAddr g_static_addr[kMaxDevices];
 
-// Device address of the array on device `dev`, which is current.  Looked up once.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id of the current context (0 if it cannot be read).
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur == nullptr || get_id == nullptr || get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of the array on device `dev`, which is current: looked up once per
+// device and context (cudaGetSymbolAddress), then reused.
 muon_status_t static_scratch(int dev, void** addr) {
   if (dev < 0 || dev >= kMaxDevices) return MUON_ERR_NO_DEVICE;
   std::lock_guard<std::mutex> lk(g_static_mu);
-  if (g_static_addr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  StaticAddr& e = g_static_addr[dev];
+  if (e.addr == nullptr || ctx == 0 || e.ctx_id != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return MUON_ERR_CUDA;
-    g_static_addr[dev] = p;
+    e.addr = p;
+    e.ctx_id = ctx;
   }
-  *addr = g_static_addr[dev];
+  *addr = e.addr;
   return MUON_OK;
 }
 

@@ -38,10 +38,21 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.muon_abi_version() == _lib.MUON_ABI_VERSION == 3
-    for code in range(9):
+    assert L.muon_abi_version() == _lib.MUON_ABI_VERSION == 4
+    for code in range(11):
         assert L.muon_status_str(code).decode() not in ("", "unknown status")
     assert L.muon_status_str(99).decode() == "unknown status"
+
+
+def test_status_codes_match_the_header():
+    import re
+
+    with open(os.path.join(ROOT, "include", "muon_b200.h")) as f:
+        text = f.read()
+    codes = {k: int(v) for k, v in re.findall(r"\b(MUON_(?:OK|ERR_[A-Z_]+))\s*=\s*(\d+)", text)}
+    assert codes["MUON_ERR_NONFINITE"] == 10
+    for name, value in codes.items():
+        assert getattr(_lib, name) == value, name
 
 
 def mats_of(shapes, base=1 << 40, dtype=_lib.MUON_BF16, spacing=1 << 34):

@@ -83,16 +83,36 @@ def test_strided_views_match_contiguous():
         assert torch.count_nonzero(b[:, :8]).item() == 0 and torch.count_nonzero(b[:, 8 + W.shape[1]:]).item() == 0
 
 
-def test_nan_stays_in_its_matrix():
+def test_nan_stays_in_its_matrix_and_is_reported():
+    """A NaN in one gradient propagates into that matrix's results only, and the
+    elementwise pass reports it: MUON_ERR_NONFINITE with the matrix's index, and the count
+    of non-finite u (u = g + beta (beta m + g) is non-finite exactly where g or m is)."""
     require_gpu()
-    from newton_schulz_11_b200 import api
+    from newton_schulz_11_b200 import _lib, api
 
-    Ws, gs, ms = _set([(128, 128), (128, 256)], dtype=torch.float32)
-    gs[0][3, 5] = float("nan")
+    Ws, gs, ms = _set([(128, 128), (128, 256), (200, 72)], dtype=torch.float32)
+    ws = api.Workspace(gs[0].device)
     O = [torch.empty_like(g) for g in gs]
-    api.muon_step(Ws, gs, ms, lr=0.02, outs=O)
-    assert torch.isnan(O[0]).any()
-    assert torch.isfinite(O[1]).all() and torch.isfinite(Ws[1]).all()
+    api.muon_step(Ws, gs, ms, lr=0.02, outs=O, workspace=ws)
+    assert api.device_status(ws) == (_lib.MUON_OK, 0)
+    assert api.nonfinite_count(ws) == 0
+    gs[1][3, 5] = float("nan")
+    gs[1][100, 7] = float("inf")
+    ms[1][0, 255] = float("-inf")
+    api.muon_step(Ws, gs, ms, lr=0.02, outs=O, workspace=ws)
+    assert torch.isnan(O[1]).any()
+    for i in (0, 2):
+        assert torch.isfinite(O[i]).all() and torch.isfinite(Ws[i]).all() and torch.isfinite(ms[i]).all()
+    assert api.device_status(ws) == (_lib.MUON_ERR_NONFINITE, 1)
+    assert api.nonfinite_count(ws) == 3
+    # sticky until cleared; Newton-Schulz alone checks its input G the same way
+    api.clear_device_status(ws)
+    assert api.device_status(ws) == (_lib.MUON_OK, 0) and api.nonfinite_count(ws) == 0
+    G = [torch.randn(96, 64, device="cuda"), torch.randn(64, 64, device="cuda")]
+    G[1][7, 7] = float("nan")
+    api.newton_schulz(G, workspace=ws)
+    assert api.device_status(ws) == (_lib.MUON_ERR_NONFINITE, 1)
+    assert api.nonfinite_count(ws) == 1
 
 
 def test_checkpoint_round_trip_is_bit_identical():
