@@ -4,10 +4,13 @@ in one grouped call (momentum, Nesterov input, Frobenius norm, 5 Newton-Schulz
 iterations, fused parameter update), timed with CUDA events.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--parallel single|sharded|replicas]
 
-Prints one JSON line (rank 0).  Under torchrun every rank steps its own copy of the
-parameter set (weak scaling, no collective on the data path); the step time is the
-maximum over ranks.
+Prints one JSON line (rank 0).  Under torchrun the default is the sharded data-parallel
+step: each matrix is stepped on one owner rank (gradients averaged onto the owners, the
+updated parameters broadcast back), so the whole job's work is fixed as N grows (strong
+scaling) and the step time is the maximum over ranks.  `--parallel replicas` instead runs
+an independent copy of the whole step on every rank (weak scaling).
 """
 from __future__ import annotations
 
@@ -31,7 +34,10 @@ if ROOT not in sys.path:
 from newton_schulz_11_b200 import inputs  # noqa: E402
 
 DEFAULT_WORKLOAD = "gpt2-124m-72-matrices"
+WIDE_WORKLOAD = "wide-4096-192-matrices"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# spec-sheet figures of one B200: HBM3e bandwidth and dense (not 2:4 sparse) bf16 tensor peak
+NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 KINDS = ("momentum", "norm", "gram", "poly", "apply", "apply_last")
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture of
@@ -203,6 +209,92 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(use), "samples_in_timed_region": len(inside)}
 
 
+class NvmlSampler:
+    """SM clock and clock-event reasons sampled in-process by NVML every `period` seconds on a
+    thread, so that a timed region of a few tens of milliseconds still holds samples (the
+    nvidia-smi loop above cannot sample faster than every few tens of milliseconds)."""
+
+    REASONS = (("sw_power_cap", 0x4), ("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20),
+               ("hw_thermal_slowdown", 0x40), ("hw_power_brake_slowdown", 0x80))
+
+    def __init__(self, device_index, period=0.002):
+        self.period = period
+        self.samples = []
+        self.t0 = self.t1 = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.handle = None
+        self.max_mhz = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(gpu_id_for(device_index))
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+        except Exception:  # pragma: no cover - depends on the machine
+            self.handle = None
+
+    def _loop(self):
+        nv, h = self.nv, self.handle
+        while not self._stop.is_set():
+            t = time.perf_counter()
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                why = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+            except Exception:  # pragma: no cover
+                break
+            self.samples.append((t, sm, why))
+            time.sleep(self.period)
+
+    def start(self):
+        if self.handle is not None:
+            self._thread = threading.Thread(target=self._loop, daemon=True)
+            self._thread.start()
+
+    def mark(self, begin: bool):
+        if begin:
+            self.t0 = time.perf_counter()
+        else:
+            self.t1 = time.perf_counter()
+
+    def stop(self):
+        if self._thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"], "samples": 0}
+        self._stop.set()
+        self._thread.join(timeout=5)
+        inside = [x for x in self.samples if self.t0 is not None and self.t1 is not None and self.t0 <= x[0] <= self.t1]
+        sm = [x[1] for x in inside]
+        reasons = sorted({name for _, _, why in inside for name, bit in self.REASONS if why & bit})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples_in_timed_region": len(inside), "period_ms": self.period * 1e3, "source": "nvml"}
+
+
+class Clocks:
+    """Both samplers around one timed region: NVML in-process (the record used, every 2 ms)
+    and the nvidia-smi loop of the profiling recipe (kept beside it)."""
+
+    def __init__(self, device_index):
+        self.nvml = NvmlSampler(device_index)
+        self.smi = ClockSampler(gpu_id_for(device_index))
+
+    def start(self):
+        self.smi.start()
+        self.nvml.start()
+
+    def mark(self, begin: bool):
+        self.nvml.mark(begin)
+        self.smi.mark(begin)
+
+    def stop(self):
+        rec = self.nvml.stop()
+        smi = self.smi.stop()
+        if rec.get("samples_in_timed_region", 0) == 0:  # no NVML: fall back on nvidia-smi's record
+            rec = dict(smi, source="nvidia-smi")
+        rec["nvidia_smi"] = smi
+        return rec
+
+
 def gpu_id_for(device_index):
     import torch
 
@@ -214,34 +306,82 @@ def gpu_id_for(device_index):
 
 # ------------------------------------------------------------------ CPU oracle timing
 
-def oracle_sample_ms(w, reps=1):
-    """Times the fp64 oracle on one matrix of each distinct shape and scales by the count
-    of that shape: milliseconds per full step (extrapolated), plus the sample description."""
-    import numpy as np
+class OracleWorkload:
+    """The fp64 oracle on the host cores over a workload's matrices: the same seeded draws
+    as the GPU arm's, made on the host once per matrix and cached."""
 
-    import oracle
+    def __init__(self, w):
+        import numpy as np
 
-    coeffs = load_coeffs(w)
-    shapes = {}
-    for i, s in enumerate(w.shapes):
-        shapes.setdefault(s, []).append(i)
-    total_ms = 0.0
-    for s, idx in shapes.items():
-        i = idx[0]
-        step = inputs.first_step_index(w)
-        g = inputs.grad_np(w, step, i).astype(np.float64)
-        m = inputs.momentum_np(w, i).astype(np.float64)
-        W = inputs.weight_np(w, i).astype(np.float64)
-        best = float("inf")
-        for _ in range(reps):
-            t0 = time.perf_counter()
-            oracle.muon_step(W, g, m, lr=w.lr, beta=w.beta, weight_decay=w.weight_decay,
-                             nesterov=w.nesterov, coeffs=coeffs)
-            best = min(best, time.perf_counter() - t0)
-        total_ms += best * 1e3 * len(idx)
-    sample = (f"one matrix of each of the {len(shapes)} shapes of {w.name} through the fp64 oracle "
-              f"(momentum, NS x{w.ns_steps}, update), time scaled by the count of each shape")
-    return total_ms, sample
+        import oracle
+
+        self.np, self.oracle = np, oracle
+        self.w = w
+        self.coeffs = load_coeffs(w)
+        self.step = inputs.first_step_index(w)
+        self.cache = {}
+
+    def work(self, i):
+        r, c = self.w.shapes[i]
+        mw = matrix_work(r, c)
+        return (mw["gram"] + mw["poly"] + mw["apply"]) * self.w.ns_steps + 16 * r * c
+
+    def data(self, i):
+        if i not in self.cache:
+            f64 = self.np.float64
+            self.cache[i] = (inputs.weight_np(self.w, i).astype(f64), inputs.grad_np(self.w, self.step, i).astype(f64),
+                             inputs.momentum_np(self.w, i).astype(f64))
+        return self.cache[i]
+
+    def run(self, idx):
+        """Seconds the oracle's step (momentum, Newton-Schulz, update) takes on matrices idx."""
+        w = self.w
+        data = [self.data(i) for i in idx]
+        t0 = time.perf_counter()
+        for W, g, m in data:
+            self.oracle.muon_step(W, g, m, lr=w.lr, beta=w.beta, weight_decay=w.weight_decay, nesterov=w.nesterov,
+                                  coeffs=self.coeffs)
+        return time.perf_counter() - t0
+
+    def plan(self, runs, budget_s):
+        """Matrices per run so that `runs` runs take about budget_s: the whole workload when it
+        fits, else a window of consecutive matrices (taken cyclically), scaled to the whole
+        workload by work.  Returns (list of index lists, total work, description)."""
+        n = len(self.w.shapes)
+        per_shape = {}
+        for i, s in enumerate(self.w.shapes):
+            if s not in per_shape:
+                per_shape[s] = self.run([i]) / max(1, self.work(i))
+        est = [per_shape[s] * self.work(i) for i, s in enumerate(self.w.shapes)]
+        total = sum(self.work(i) for i in range(n))
+        if runs * sum(est) <= budget_s:
+            return [list(range(n))] * runs, total, f"the full step: all {n} matrices of {self.w.name}"
+        per_run = budget_s / runs
+        plans, start = [], 0
+        for _ in range(runs):
+            idx, t = [], 0.0
+            while not idx or (t + est[start % n] <= per_run and len(idx) < n):
+                idx.append(start % n)
+                t += est[start % n]
+                start += 1
+            plans.append(idx)
+        k = max(len(p) for p in plans)
+        return plans, total, (f"per run up to {k} consecutive matrices of {self.w.name} (cyclically), "
+                              f"scaled to all {n} by algorithmic work, to keep the run within {budget_s:.0f} s")
+
+    def ms_per_step(self, idx, total):
+        return self.run(idx) * 1e3 * total / sum(self.work(i) for i in idx)
+
+
+def oracle_baseline_ms(w, budget_s=30.0):
+    """cpu_baseline of the GPU arm: the oracle on one step of the workload (the whole step
+    when it takes at most budget_s), best of two runs when they fit."""
+    ow = OracleWorkload(w)
+    plans, total, sample = ow.plan(1, budget_s)
+    runs = [ow.ms_per_step(plans[0], total)]
+    if runs[0] * 2e-3 <= budget_s:
+        runs.append(ow.ms_per_step(plans[0], total))
+    return min(runs), sample + (f", best of {len(runs)}" if len(runs) > 1 else "")
 
 
 def blas_threads():
@@ -314,71 +454,200 @@ def workload_of(args):
     return w
 
 
-def oracle_step_samples(w):
-    """One bounded sample per reference step: the fp64 oracle's step on ONE matrix,
-    cycling through the workload's distinct shapes; each sample is scaled to a full step
-    by the work ratio (algorithmic NS flops plus elementwise elements) of the whole
-    workload to that matrix.  Yields (ms per full step, shape)."""
-    import numpy as np
+def parallel_mode(args, world):
+    mode = getattr(args, "parallel", None)
+    if mode in (None, "auto"):
+        mode = "sharded" if world > 1 else "single"
+    if mode == "single" and world > 1:
+        mode = "replicas"
+    return mode
 
-    import oracle
 
-    coeffs = load_coeffs(w)
-    by_shape = {}
-    for i, s in enumerate(w.shapes):
-        by_shape.setdefault(s, []).append(i)
+def config_of(w, world, mode):
+    """The `config` object both arms print for a workload."""
+    return {"workload": w.name, "matrices": len(w.shapes), "params": w.n_params, "param_dtype": w.param_dtype,
+            "ns_steps": w.ns_steps, "schedule": w.schedule,
+            "l2": "inputs larger than L2 (grads+momentum+params ~%.2f GB)" % (w.n_params * 10 / 1e9),
+            "parallelism": mode if world > 1 else "single"}
 
-    def work(r, c):
-        mw = matrix_work(r, c)
-        return (mw["gram"] + mw["poly"] + mw["apply"]) * w.ns_steps + 16 * r * c
 
-    total = sum(work(r, c) for r, c in w.shapes)
-    shapes = list(by_shape)
-    step = inputs.first_step_index(w)
-    cache = {}
-    k = 0
-    while True:
-        s = shapes[k % len(shapes)]
-        k += 1
-        if s not in cache:
-            i = by_shape[s][0]
-            cache[s] = tuple(x.astype(np.float64) for x in (inputs.weight_np(w, i), inputs.grad_np(w, step, i),
-                                                              inputs.momentum_np(w, i)))
-        W, g, m = cache[s]
-        t0 = time.perf_counter()
-        oracle.muon_step(W, g, m, lr=w.lr, beta=w.beta, weight_decay=w.weight_decay, nesterov=w.nesterov,
-                         coeffs=coeffs)
-        dt = time.perf_counter() - t0
-        yield dt * 1e3 * total / work(*s), s
+REFERENCE_BUDGET_S = 150.0
 
 
 def run_reference(args, world, rank):
-    """The oracle, as it stands, on the host cores.  Each step is one bounded sample (one
-    matrix, shapes taken in turn) scaled to a full step; value = median over the steps."""
+    """The oracle, as it stands, on the host cores: each of the W + K steps runs the oracle's
+    step over the workload (all of it when W + K full steps fit in about REFERENCE_BUDGET_S,
+    else a window of matrices scaled to the whole step by work); value = median over K."""
     if rank != 0:
         return
     w = workload_of(args)
-    gen = oracle_step_samples(w)
-    for _ in range(args.warmup):
-        next(gen)
-    runs = [next(gen) for _ in range(args.steps)]
-    value = statistics.median(r[0] for r in runs)
+    ow = OracleWorkload(w)
+    plans, total, sample = ow.plan(args.warmup + args.steps, getattr(args, "budget_s", REFERENCE_BUDGET_S))
+    for idx in plans[:args.warmup]:
+        ow.run(idx)
+    runs = [ow.ms_per_step(idx, total) for idx in plans[args.warmup:]]
+    value = statistics.median(runs)
     cores = blas_threads()
-    sample = (f"per step: the fp64 oracle (momentum, NS x{w.ns_steps}, update) on one matrix of {w.name}, "
-              f"the {len(set(w.shapes))} shapes in turn, scaled to the full step by work ratio; "
-              f"median of {args.steps} steps")
+    mode = parallel_mode(args, world)
     line = {
         "impl": "reference", "metric": "muon_step_ms", "value": round(value, 3), "unit": "ms",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(value, 3),
-        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": w.name, "matrices": len(w.shapes), "params": w.n_params},
-        "cpu_baseline": {"value": round(value, 3), "unit": "ms", "cores": cores, "kind": "oracle", "sample": sample},
+        "higher_is_better": False, "scaling": "weak" if mode == "replicas" else "strong", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic", "config": config_of(w, world, mode),
+        "cpu_baseline": {"value": round(value, 3), "unit": "ms", "cores": cores, "kind": "oracle",
+                         "sample": f"{sample}; median of {args.steps} steps after {args.warmup} warm-up steps"},
         "e2e": {"value": round(value, 3), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
 # ------------------------------------------------------------------ our arm
+
+def roofline_of(flops, nbytes, ms, peaks, peak_src):
+    """Roofline of one kernel from its algorithmic work per launch and its mean launch time.
+    The binding bound is the one whose floor time (work / peak) is the longer; `frac` is that
+    floor over the measured time.  The tensor denominator is the measured burst bf16 peak,
+    fixed whatever the clocks did; the power-capped sustained peak and the spec-sheet figures
+    are reported beside it."""
+    t = ms * 1e-3
+    tf = flops / t / 1e12 if flops else 0.0
+    gbs = nbytes / t / 1e9
+    f_t = tf / peaks["bf16_tflops"]
+    f_h = gbs / peaks["hbm_gbs"]
+    tensor = flops > 0 and f_t >= f_h
+    return {"bound": "tensor" if tensor else "hbm", "achieved": round(tf if tensor else gbs, 1),
+            "peak": peaks["bf16_tflops"] if tensor else peaks["hbm_gbs"], "unit": "TFLOP/s" if tensor else "GB/s",
+            "frac": round(max(f_t, f_h), 4),
+            "peak_source": f"{peak_src} {'burst bf16 GEMM' if tensor else 'copy bandwidth'}",
+            "frac_tensor": round(f_t, 4), "frac_hbm": round(f_h, 4),
+            "frac_tensor_of_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
+            "frac_nominal": {"tensor": round(tf / NOMINAL_PEAKS["bf16_tflops"], 4),
+                             "hbm": round(gbs / NOMINAL_PEAKS["hbm_gbs"], 4)},
+            "achieved_tflops": round(tf, 1), "achieved_gbs": round(gbs, 1),
+            "algorithmic_flops_per_launch": int(flops), "algorithmic_bytes_per_launch": int(nbytes),
+            "ms_per_launch": round(ms, 4)}
+
+
+def make_step(w, ps, gs, ms, *, mode, world, waves=2, workspace=None, local_step=None):
+    """The step the bench times: one PreparedMuonStep over every matrix (single, replicas), or
+    the sharded data-parallel step (ShardedMuon: gradients averaged onto each matrix's owner,
+    the owners' grouped steps, parameters broadcast back).  Returns (step(), owned indices)."""
+    hyper = dict(lr=w.lr, beta=w.beta, weight_decay=w.weight_decay, nesterov=w.nesterov, coeffs=load_coeffs(w))
+    if mode == "sharded":
+        from newton_schulz_11_b200.distributed import ShardedMuon
+
+        if workspace is not None:
+            hyper["workspace"] = workspace
+        sh = ShardedMuon(ps, gs, ms, reduce_grads=world > 1, waves=waves, local_step=local_step, **hyper)
+        return sh, list(sh.owned)
+    from newton_schulz_11_b200 import api
+
+    fn = api.PreparedMuonStep(ps, gs, ms, workspace=workspace, **hyper)
+    return (lambda: fn()), list(range(len(ps)))
+
+
+def time_steps(step, steps, world, device):
+    """Milliseconds per step over `steps` steps, bracketed by a barrier and a device
+    synchronisation on both sides, timed on the device (CUDA events on the current stream;
+    wall clock for CPU ranks); the max over ranks."""
+    import torch
+
+    cuda = torch.device(device).type == "cuda"
+    barrier(world)
+    if cuda:
+        torch.cuda.synchronize(device)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            step()
+        e1.record()
+        torch.cuda.synchronize(device)
+        ms = e0.elapsed_time(e1) / steps
+    else:
+        t0 = time.perf_counter()
+        for _ in range(steps):
+            step()
+        ms = (time.perf_counter() - t0) * 1e3 / steps
+    barrier(world)
+    return dist_max(ms, world)
+
+
+def base_line(w, world, mode, ms_step, args):
+    """The contract's keys of our arm's JSON line."""
+    return {"metric": "muon_step_ms", "value": round(ms_step, 4), "unit": "ms", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": False,
+            "scaling": "weak" if mode == "replicas" else "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": config_of(w, world, mode)}
+
+
+def flat_workload(w, dev, step):
+    """The workload's grads, momentum and params in three flat device buffers, one 2-D view
+    per matrix (so that the host copies of e2e are one copy each)."""
+    import torch
+
+    sizes = [r * c for r, c in w.shapes]
+    offs = [0]
+    for n in sizes:
+        offs.append(offs[-1] + n)
+    pdt = torch.bfloat16 if w.param_dtype == "bf16" else torch.float32
+    G = torch.empty(offs[-1], dtype=torch.float32, device=dev)
+    M = torch.empty(offs[-1], dtype=torch.float32, device=dev)
+    P = torch.empty(offs[-1], dtype=pdt, device=dev)
+    views = lambda flat: [flat[offs[i]: offs[i + 1]].view(*w.shapes[i]) for i in range(len(sizes))]  # noqa: E731
+    gs, ms, ps = views(G), views(M), views(P)
+    with torch.no_grad():
+        for i in range(len(sizes)):
+            gs[i].copy_(inputs.grad_torch(w, step, i, dev))
+            ms[i].copy_(inputs.momentum_torch(w, i, dev))
+            ps[i].copy_(inputs.weight_torch(w, i, dev))
+    torch.cuda.synchronize(dev)
+    return (G, M, P), (gs, ms, ps), views
+
+
+def measure_wide(local, peaks, peak_src, steps=5, warmup=3):
+    """The 4096-wide set (192 matrices, 5.9B parameters) on this GPU, inputs drawn on the
+    device: step time, Newton-Schulz TFLOP/s and its fractions, with the clocks of its own
+    timed region."""
+    import torch
+
+    from newton_schulz_11_b200 import api
+
+    dev = torch.device("cuda", local)
+    w = inputs.WORKLOADS[WIDE_WORKLOAD]
+    free, _ = torch.cuda.mem_get_info(dev)
+    need = w.n_params * 10 + api.workspace_size(w.shapes)
+    if free < need * 1.1:
+        return {"skipped": f"needs {need / 1e9:.0f} GB, {free / 1e9:.0f} GB free"}
+    _, (gs, ms, ps), _ = flat_workload(w, dev, inputs.first_step_index(w))
+    ws = api.Workspace(dev)
+    step, _ = make_step(w, ps, gs, ms, mode="single", world=1, workspace=ws)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    clocks = Clocks(local)
+    clocks.start()
+    clocks.mark(True)
+    ms_step = time_steps(step, steps, 1, dev)
+    clocks.mark(False)
+    clk = clocks.stop()
+    code, where = api.device_status(ws)
+    if code != 0:
+        raise RuntimeError(f"device status {code} at {where} in the 4096-wide run")
+    alg, dense = step_flops(w)
+    tf = alg / (ms_step * 1e-3) / 1e12
+    out = {"workload": w.name, "matrices": len(w.shapes), "params": w.n_params, "ms_per_step": round(ms_step, 2),
+           "steps": steps, "warmup": warmup, "ns_tflops": round(tf, 1),
+           "ns_tflops_dense_equiv": round(dense / (ms_step * 1e-3) / 1e12, 1),
+           "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
+           "frac_of_bf16_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
+           "frac_of_nominal_bf16": round(tf / NOMINAL_PEAKS["bf16_tflops"], 4),
+           "peak_source": peak_src, "clocks": clk,
+           "note": "whole step (elementwise pass included) timed; NS flops over the step time"}
+    del gs, ms, ps, step, ws
+    torch.cuda.empty_cache()
+    return out
+
 
 def run_ours(args, world, rank, local):
     import ctypes
@@ -391,59 +660,29 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     w = workload_of(args)
-    coeffs = load_coeffs(w)
+    mode = parallel_mode(args, world)
     step0 = inputs.first_step_index(w)
-
-    # flat device buffers with one 2-D view per matrix (one H2D / D2H copy per step in e2e)
-    sizes = [r * c for r, c in w.shapes]
-    offs = [0]
-    for s in sizes:
-        offs.append(offs[-1] + s)
-    pdt = torch.bfloat16 if w.param_dtype == "bf16" else torch.float32
-    G = torch.empty(offs[-1], dtype=torch.float32, device=dev)
-    M = torch.empty(offs[-1], dtype=torch.float32, device=dev)
-    P = torch.empty(offs[-1], dtype=pdt, device=dev)
-    view = lambda flat, i: flat[offs[i]: offs[i + 1]].view(*w.shapes[i])  # noqa: E731
-    gs = [view(G, i) for i in range(len(sizes))]
-    ms = [view(M, i) for i in range(len(sizes))]
-    ps = [view(P, i) for i in range(len(sizes))]
-    with torch.no_grad():
-        for i in range(len(sizes)):
-            gs[i].copy_(inputs.grad_torch(w, step0, i, dev))
-            ms[i].copy_(inputs.momentum_torch(w, i, dev))
-            ps[i].copy_(inputs.weight_torch(w, i, dev))
-    torch.cuda.synchronize()
-
+    (G, M, P), (gs, ms, ps), views = flat_workload(w, dev, step0)
     ws = api.Workspace(dev)
     stream = torch.cuda.current_stream(dev)
-    # the descriptors are built once (PreparedMuonStep); every step is one C ABI call
-    step_fn = api.PreparedMuonStep(ps, gs, ms, lr=w.lr, beta=w.beta, weight_decay=w.weight_decay,
-                                   nesterov=w.nesterov, coeffs=coeffs, workspace=ws)
+    step, owned = make_step(w, ps, gs, ms, mode=mode, world=world, waves=args.waves, workspace=ws)
+    # the kernels of this rank run on its own matrices (all of them unless sharded)
+    w_local = w if len(owned) == len(w.shapes) else inputs.scaled_workload(
+        w, [w.shapes[i] for i in owned], name=f"{w.name}[owned by rank {rank}]")
 
     for _ in range(args.warmup):
-        step_fn(stream)
+        step()
     torch.cuda.synchronize()
 
     L = _lib.lib()
-    clocks = ClockSampler(gpu_id_for(local))
+    clocks = Clocks(local)
     clocks.start()
     # ---- timed region: K steps, inputs resident in HBM (larger than L2).  No per-kernel
     # events here: an event between two launches would stop their programmatic overlap.
-    barrier(world)
-    torch.cuda.synchronize()
     clocks.mark(True)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        step_fn(stream)
-    e1.record(stream)
-    torch.cuda.synchronize()
+    ms_step = time_steps(step, args.steps, world, dev)
     clocks.mark(False)
-    barrier(world)
-    ms_step = e0.elapsed_time(e1) / args.steps
     clk = clocks.stop()
-    ms_step = dist_max(ms_step, world)
 
     # ---- step-time spread: events between steps only (launches inside a step keep their
     # programmatic overlap); p10 / p50 / p90 over up to 200 steps
@@ -452,7 +691,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     evs[0].record(stream)
     for i in range(spread_steps):
-        step_fn(stream)
+        step()
         evs[i + 1].record(stream)
     torch.cuda.synchronize()
     per_step = sorted(evs[i].elapsed_time(evs[i + 1]) for i in range(spread_steps))
@@ -465,7 +704,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     _lib.check(L.muon_profile_begin(), "muon_profile_begin")
     for _ in range(prof_steps):
-        step_fn(stream)
+        step()
     torch.cuda.synchronize()
     kms = (ctypes.c_double * 6)()
     kcount = (ctypes.c_int64 * 6)()
@@ -473,63 +712,10 @@ def run_ours(args, world, rank, local):
     launches_per_step = sum(kcount) // prof_steps
 
     # ---- end to end through host buffers: every step copies its grads in from pinned host
-    # memory and its params out to pinned host memory.  Pipelined over two copy streams:
-    # step t + 1's grads come in (into the other of two grad buffers) and step t's params
-    # go out (from a device snapshot taken right after the step) while step t + 1 runs.
+    # memory and its params out to pinned host memory.
     e2e_ms = None
     if not args.no_e2e:
-        G2 = torch.empty_like(G)
-        step_fn2 = api.PreparedMuonStep(ps, [view(G2, i) for i in range(len(sizes))], ms, lr=w.lr, beta=w.beta,
-                                        weight_decay=w.weight_decay, nesterov=w.nesterov, coeffs=coeffs,
-                                        workspace=ws)
-        gbuf, steps_fn = (G, G2), (step_fn, step_fn2)
-        snap = (torch.empty_like(P), torch.empty_like(P))
-        pin_g = torch.empty_like(G, device="cpu").pin_memory()
-        pin_g.copy_(G.cpu())
-        pin_p = (torch.empty_like(P, device="cpu").pin_memory(), torch.empty_like(P, device="cpu").pin_memory())
-        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        ev = lambda: torch.cuda.Event()  # noqa: E731
-
-        def run_e2e(n):
-            in_done, step_done, out_done = [None, None], [None, None], [None, None]
-            for t in range(n):
-                b = t % 2
-                if step_done[b] is not None:
-                    s_in.wait_event(step_done[b])      # the step that read this grad buffer is done
-                with torch.cuda.stream(s_in):
-                    gbuf[b].copy_(pin_g, non_blocking=True)
-                in_done[b] = ev()
-                in_done[b].record(s_in)
-                stream.wait_event(in_done[b])
-                steps_fn[b](stream)
-                if out_done[b] is not None:
-                    stream.wait_event(out_done[b])     # the snapshot's previous copy-out is done
-                snap[b].copy_(P, non_blocking=True)
-                step_done[b] = ev()
-                step_done[b].record(stream)
-                s_out.wait_event(step_done[b])
-                with torch.cuda.stream(s_out):
-                    pin_p[b].copy_(snap[b], non_blocking=True)
-                out_done[b] = ev()
-                out_done[b].record(s_out)
-            for e in out_done:
-                if e is not None:
-                    stream.wait_event(e)
-
-        run_e2e(2)
-        torch.cuda.synchronize()
-        barrier(world)
-        f0 = torch.cuda.Event(enable_timing=True)
-        f1 = torch.cuda.Event(enable_timing=True)
-        e2e_steps = max(2, min(args.steps, 50))
-        f0.record(stream)
-        s_in.wait_event(f0)
-        s_out.wait_event(f0)
-        run_e2e(e2e_steps)
-        f1.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = dist_max(f0.elapsed_time(f1) / e2e_steps, world)
-        barrier(world)
+        e2e_ms = run_e2e(w, mode, world, step, (G, M, P), (gs, ms, ps), views, ws, stream, args)
 
     code, where = api.device_status(ws)
     if code != 0:
@@ -545,51 +731,41 @@ def run_ours(args, world, rank, local):
     # their summed time (a workload of several waves has several launches per iteration).
     iters = {"momentum": 1, "norm": 1, "gram": w.ns_steps, "poly": w.ns_steps, "apply": w.ns_steps - 1,
              "apply_last": 1}
-    dom_launches = max(1, per_kind[dom]["launches"])
-    dom_ms = per_kind[dom]["ms_total"] / dom_launches
-    fl = kind_flops(w, dom) * iters[dom] * prof_steps / dom_launches    # per launch (mean)
-    by = kind_bytes(w, dom) * iters[dom] * prof_steps / dom_launches
-    tf = fl / (dom_ms * 1e-3) / 1e12 if fl else 0.0
-    gbs = by / (dom_ms * 1e-3) / 1e9
-    # a tensor-bound kernel timed while the power cap held the clocks takes the sustained peak
-    capped = "sw_power_cap" in (clk.get("reasons") or [])
-    tpeak_key = "bf16_tflops_sustained" if capped else "bf16_tflops"
-    f_tensor = tf / peaks[tpeak_key] if fl else 0.0
-    f_hbm = gbs / peaks["hbm_gbs"]
+
+    def per_launch(kind):
+        n = max(1, per_kind[kind]["launches"])
+        return (kind_flops(w_local, kind) * iters[kind] * prof_steps / n,
+                kind_bytes(w_local, kind) * iters[kind] * prof_steps / n, per_kind[kind]["ms_total"] / n)
+
+    fl, by, dom_ms = per_launch(dom)
+    roof = roofline_of(fl, by, dom_ms, peaks, peak_src)
     traffic = None
-    if NCU_TRAFFIC["source_hash"] == kernel_source_hash() and NCU_TRAFFIC["workload"] == w.name:
+    if NCU_TRAFFIC["source_hash"] == kernel_source_hash() and NCU_TRAFFIC["workload"] == w_local.name:
         traffic = NCU_TRAFFIC["bytes_per_launch"].get(dom)
-    if f_tensor >= f_hbm:
-        roof = {"bound": "tensor", "achieved": round(tf, 1), "peak": peaks[tpeak_key], "unit": "TFLOP/s",
-                "frac": round(f_tensor, 4)}
-    else:
-        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(f_hbm, 4)}
-    roof.update({"traffic": traffic, "kernel": dom,
-                 "peak_source": peak_src + (" sustained (power cap active)" if capped and roof["bound"] == "tensor"
-                                            else " burst" if roof["bound"] == "tensor" else " copy"),
-                 "other_bound_frac": round(min(f_tensor, f_hbm), 4),
-                 "algorithmic_bytes_per_launch": int(by), "algorithmic_flops_per_launch": int(fl),
-                 "ms_per_launch": round(dom_ms, 4)})
+    roof = {**{k: roof[k] for k in ("bound", "achieved", "peak", "unit", "frac")}, "traffic": traffic,
+            "kernel": dom, **{k: v for k, v in roof.items() if k not in ("bound", "achieved", "peak", "unit", "frac")}}
+    _, ew_by, ew_ms = per_launch("momentum")
+    ew = roofline_of(0, ew_by, ew_ms, peaks, peak_src)
 
     alg, dense = step_flops(w)
-    line = {
-        "metric": "muon_step_ms", "value": round(ms_step, 4), "unit": "ms", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic",
-        "config": {"workload": w.name, "matrices": len(w.shapes), "params": w.n_params,
-                   "param_dtype": w.param_dtype, "ns_steps": w.ns_steps, "schedule": w.schedule,
-                   "l2": "inputs larger than L2 (grads+momentum+params ~%.2f GB)" % (w.n_params * 10 / 1e9),
-                   "parallelism": "replicas" if world > 1 else "single"},
-        "ns_tflops": round(world * alg / (ms_step * 1e-3) / 1e12, 1),
-        "ns_tflops_dense_equiv": round(world * dense / (ms_step * 1e-3) / 1e12, 1),
-        "ns_frac_of_bf16_peak": round(alg / (ms_step * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
-        "ns_frac_of_bf16_sustained": round(alg / (ms_step * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"], 4),
+    jobs = world if mode == "replicas" else 1  # whole-job work per step
+    tf = jobs * alg / (ms_step * 1e-3) / 1e12
+    line = base_line(w, world, mode, ms_step, args)
+    line.update({
+        "ns_tflops": round(tf, 1),
+        "ns_tflops_dense_equiv": round(jobs * dense / (ms_step * 1e-3) / 1e12, 1),
+        # per GPU: the whole job's Newton-Schulz flops over the step time, over N GPUs' peaks
+        "ns_frac_of_bf16_peak": round(tf / world / peaks["bf16_tflops"], 4),
+        "ns_frac_of_bf16_sustained": round(tf / world / peaks["bf16_tflops_sustained"], 4),
+        "ns_frac_of_nominal_bf16": round(tf / world / NOMINAL_PEAKS["bf16_tflops"], 4),
         "kernels": {k: {"ms_per_launch": round(v["ms_total"] / max(1, v["launches"]), 4),
                         "launches": v["launches"], "share": round(v["ms_total"] / max(1e-9, sum(
                             x["ms_total"] for x in per_kind.values())), 4)} for k, v in per_kind.items()},
         "roofline": roof,
+        "elementwise": {"kernel": "muon_momentum_kernel", "achieved_gbs": ew["achieved_gbs"],
+                        "frac_of_measured_hbm": ew["frac_hbm"], "frac_of_nominal_hbm": ew["frac_nominal"]["hbm"],
+                        "algorithmic_bytes_per_launch": ew["algorithmic_bytes_per_launch"],
+                        "ms_per_launch": ew["ms_per_launch"]},
         "clocks": clk,
         "e2e": None if e2e_ms is None else {
             "value": round(e2e_ms, 4), "unit": "ms", "h2d_bytes_per_step": G.numel() * 4,
@@ -597,12 +773,100 @@ def run_ours(args, world, rank, local):
         "gpu_launches": int(launches_per_step * args.steps),
         "profiled_steps": prof_steps,
         "ms_per_step_spread": spread,
-    }
+        "peaks": {"source": peak_src, **peaks, "nominal": NOMINAL_PEAKS},
+    })
+    if mode == "sharded" and world > 1:
+        line["sharding"] = {"owned_by_rank0": len(owned), "waves": args.waves,
+                            "collectives": "NCCL reduce of fp32 grads onto owners, broadcast of bf16 params"}
     if world == 1 and not args.no_cpu_baseline:
-        cms, sample = oracle_sample_ms(w)
+        cms, sample = oracle_baseline_ms(w)
         line["cpu_baseline"] = {"value": round(cms, 1), "unit": "ms", "cores": blas_threads(), "kind": "oracle",
                                 "sample": sample}
+    if world == 1 and w.name == DEFAULT_WORKLOAD and not args.no_wide:
+        del G, M, P, gs, ms, ps, step, ws
+        torch.cuda.empty_cache()
+        line["wide4096"] = measure_wide(local, peaks, peak_src)
     print(json.dumps(line), flush=True)
+
+
+def run_e2e(w, mode, world, step, flats, views_, view_of, ws, stream, args):
+    """Milliseconds per step through host buffers (max over ranks).  Single GPU: pipelined
+    over two copy streams -- step t + 1's grads come in (into the other of two grad
+    buffers) and step t's params go out (from a device snapshot taken right after the step)
+    while step t + 1 runs.  Sharded: every step copies its grads in, steps, and copies the
+    params out, in stream order."""
+    import torch
+
+    from newton_schulz_11_b200 import api
+
+    G, M, P = flats
+    gs, ms, ps = views_
+    dev = G.device
+    pin_g = torch.empty_like(G, device="cpu").pin_memory()
+    pin_g.copy_(G.cpu())
+    e2e_steps = max(2, min(args.steps, 50))
+    if mode == "sharded":
+        pin_p = torch.empty_like(P, device="cpu").pin_memory()
+
+        def one():
+            G.copy_(pin_g, non_blocking=True)
+            step()
+            pin_p.copy_(P, non_blocking=True)
+
+        one()
+        torch.cuda.synchronize()
+        return time_steps(one, e2e_steps, world, dev)
+
+    G2 = torch.empty_like(G)
+    coeffs = load_coeffs(w)
+    step2 = api.PreparedMuonStep(ps, view_of(G2), ms, lr=w.lr, beta=w.beta, weight_decay=w.weight_decay,
+                                 nesterov=w.nesterov, coeffs=coeffs, workspace=ws)
+    gbuf, steps_fn = (G, G2), (step, lambda: step2())
+    snap = (torch.empty_like(P), torch.empty_like(P))
+    pin_p = (torch.empty_like(P, device="cpu").pin_memory(), torch.empty_like(P, device="cpu").pin_memory())
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+
+    def run(n):
+        in_done, step_done, out_done = [None, None], [None, None], [None, None]
+        for t in range(n):
+            b = t % 2
+            if step_done[b] is not None:
+                s_in.wait_event(step_done[b])      # the step that read this grad buffer is done
+            with torch.cuda.stream(s_in):
+                gbuf[b].copy_(pin_g, non_blocking=True)
+            in_done[b] = ev()
+            in_done[b].record(s_in)
+            stream.wait_event(in_done[b])
+            steps_fn[b]()
+            if out_done[b] is not None:
+                stream.wait_event(out_done[b])     # the snapshot's previous copy-out is done
+            snap[b].copy_(P, non_blocking=True)
+            step_done[b] = ev()
+            step_done[b].record(stream)
+            s_out.wait_event(step_done[b])
+            with torch.cuda.stream(s_out):
+                pin_p[b].copy_(snap[b], non_blocking=True)
+            out_done[b] = ev()
+            out_done[b].record(s_out)
+        for e in out_done:
+            if e is not None:
+                stream.wait_event(e)
+
+    run(2)
+    torch.cuda.synchronize()
+    barrier(world)
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    s_in.wait_event(f0)
+    s_out.wait_event(f0)
+    run(e2e_steps)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    out = dist_max(f0.elapsed_time(f1) / e2e_steps, world)
+    barrier(world)
+    return out
 
 
 # ------------------------------------------------------------------ AdamW path
@@ -676,7 +940,7 @@ def run_adamw(args, world, rank, local):
         t += 1
         adamw(t, stream)
     torch.cuda.synchronize()
-    clocks = ClockSampler(gpu_id_for(local))
+    clocks = Clocks(local)
     clocks.start()
     barrier(world)
     torch.cuda.synchronize()
@@ -774,6 +1038,12 @@ def main():
                     help="muon: the Muon step (default); adamw: the AdamW step of the non-matrix parameters")
     ap.add_argument("--matrices", type=int, default=0,
                     help="run only the first K matrices of the workload (a small case of the same kernels)")
+    ap.add_argument("--parallel", default="auto", choices=["auto", "single", "sharded", "replicas"],
+                    help="N > 1: sharded data-parallel step (default) or independent replicas")
+    ap.add_argument("--waves", type=int, default=2,
+                    help="sharded: waves of owned matrices (a wave's broadcasts overlap the next wave's step)")
+    ap.add_argument("--no-wide", action="store_true",
+                    help="skip the 4096-wide measurement added to the default workload's line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
