@@ -44,9 +44,8 @@ KINDS = ("momentum", "norm", "gram", "poly", "apply", "apply_last")
 # the benchmarked workload, keyed by kernel kind; valid only while the kernel sources hash to
 # `source_hash` (kernel_source_hash: comments and layout do not count; see profiles/).
 # Filled in from the committed ncu summary.
-NCU_TRAFFIC = {"source_hash": "1bbc922b404858ed", "workload": DEFAULT_WORKLOAD,
-               "bytes_per_launch": {"momentum": 1221587712, "norm": 29952, "gram": 210905241,
-                                    "poly": 125945241, "apply": 548369472, "apply_last": 658044416}}
+NCU_TRAFFIC = {"source_hash": "62133dae96352479", "workload": DEFAULT_WORKLOAD,
+               "bytes_per_launch": {"gram": 211413760, "poly": 126011392, "apply": 550936064}}
 # the same for the AdamW path (workload gpt2-124m-adamw-params, one launch per step)
 NCU_TRAFFIC_ADAMW = {"source_hash": "1bbc922b404858ed", "bytes_per_launch": 894222080}
 
