@@ -101,12 +101,12 @@ typedef struct {
 
 /*
  * Where one matrix's scratch lives inside the workspace (diagnostics and tests).
- * X is carried between iterations as hi + lo: hi = bf16(x) (the tensor-core operand) and
- * lo = one byte per element holding the residual x - hi in fixed point.  With E' the
- * biased exponent of hi raised to at least 14 and e' = E' - 127, the residual is the
- * integer k = round-half-even((x - hi) * 2^(14 - e')), |k| <= 64 since
- * |x - hi| <= 2^(e - 8), and the stored byte is k + 64 (0 .. 128, unsigned); then
- * x = hi + k * 2^(e' - 14), within 2^(e - 15) of the fp32 value.
+ * X is carried between iterations as hi + lo: hi = bf16(x) (the tensor-core operand,
+ * rounded to nearest even) and lo = one byte per element holding the residual in fixed
+ * point on the fp32 bit patterns.  With d = bits(x) - bits(hi) as signed 32-bit integers
+ * (|d| <= 2^15, since rounding to bf16 rounds the bit pattern to a multiple of 2^16), the
+ * stored byte is (d + 2^15 + 2^8) >> 9, unsigned, 0 .. 128; x is rebuilt as the float with
+ * bits bits(hi) + 2^9 * (byte - 64), within 2^8 fp32 ulps (relative 2^-15) of the fp32 value.
  */
 typedef struct {
   uint64_t x_hi_offset[2];   /* bf16 [rows x x_ld]: ping-pong high parts of X */

@@ -372,37 +372,27 @@ __device__ __forceinline__ uint32_t float_to_bf16_bits(float x) {
 }
 
 // ---- X as hi + lo with an 8-bit lo
-// hi = bf16(x).  With E' = max(biased exponent of hi, 14) and e' = E' - 127, the residual
-// x - hi is kept as the integer k = round-half-even((x - hi) 2^(14 - e')), stored as the
-// byte k + 64, and x = hi + k 2^(e' - 14).  |x - hi| <= 2^(e - 8) bounds |k| by 64, so k
-// needs no clamp, and the residual error is at most 2^(e - 15): 15 significant bits in
-// all.  The helpers use one fma each way and byte permutes; the only integer arithmetic is
-// the exponent mask, its clamp and one subtraction.
+// hi = bf16(x), rounded to nearest even: x's fp32 bit pattern rounded to a multiple of 2^16,
+// so d = bits(x) - bits(hi), as signed 32-bit integers, lies in [-2^15, 2^15].  The stored
+// byte is (d + 2^15 + 2^8) >> 9, in 0 .. 128: d rounded to a multiple of 2^9 (halves up),
+// biased by 64.  x is rebuilt as the float whose bits are bits(hi) + 2^9 (byte - 64): within
+// 2^8 fp32 ulps of x, 15 significant bits in all.  Both ways are integer operations on the
+// bit patterns (one add and one shift to encode, one byte extraction and one shifted add to
+// decode); the residual's unit, 2^9 ulps, follows the exponent of x by construction.
 
-// 2^e' as float bits, from hi's float bits hb.
-__device__ __forceinline__ uint32_t lo8_exp_bits(uint32_t hb) { return max(hb & 0x7F800000u, 14u << 23); }
-
-// The stored byte for x against hi (float bits hb), in the low 8 bits of the result (the
-// bits above belong to 1.5 * 2^23 and are dropped by the caller): one fma scales the exact
-// residual by 2^(14 - e') (float bits 0x86000000 - 2^e' bits), rounds it to the nearest
-// integer, ties to even, and adds 1.5 * 2^23 + 64.
+// The stored byte for x against hi (float bits hb), in the low bits of the result.  The
+// unsigned sum wraps past 2^32 exactly when d < 0 and lands in [2^8, 2^16 + 2^8].
 __device__ __forceinline__ uint32_t lo8_encode_word(float x, uint32_t hb) {
-  const float r = x - __uint_as_float(hb);  // exact
-  return __float_as_uint(fmaf(r, __uint_as_float(0x86000000u - lo8_exp_bits(hb)), 12582976.f));
+  return (__float_as_uint(x) - hb + 33024u) >> 9;
 }
 
 // The stored byte for x against the bf16 hi (bit pattern in the low 16 bits).
-__device__ __forceinline__ uint32_t lo8_encode(float x, uint32_t hi16) {
-  return lo8_encode_word(x, hi16 << 16) & 0xFFu;
-}
+__device__ __forceinline__ uint32_t lo8_encode(float x, uint32_t hi16) { return lo8_encode_word(x, hi16 << 16); }
 
-// x from hi (float bits hb) and the stored byte j (0..3) of word lw: a byte permute makes
-// the float 1.5 * 2^23 + byte, one fma turns it into k 2^-14 (exact), one more adds
-// k 2^(e' - 14) to hi.
+// x from hi (float bits hb) and the stored byte j (0..3) of word lw.
 __device__ __forceinline__ float lo8_decode(uint32_t hb, uint32_t lw, uint32_t j) {
-  const float f = __uint_as_float(__byte_perm(lw, 0x4B400000u, 0x7650u | j));
-  const float k = fmaf(f, 0x1p-14f, -768.00390625f);  // (f - 1.5 * 2^23 - 64) * 2^-14
-  return fmaf(k, __uint_as_float(lo8_exp_bits(hb)), __uint_as_float(hb));
+  const uint32_t byte = __byte_perm(lw, 0u, 0x4440u | j);
+  return __uint_as_float(hb - 32768u + (byte << 9));
 }
 
 // Four values at once: hi as two bf16x2 words (h01: x0 low, x1 high; h23 likewise) and the

@@ -3,8 +3,8 @@
 //   m' = beta m + g                        ("14 - modded-nanogpt", section 3, muon_step)
 //   u  = g + beta m'  (Nesterov) or m'     ("NanoGPT Speedrun" README, practices list)
 //   hi = bf16(u), lo = 8-bit residual      Newton-Schulz input, unscaled (lo: the byte
-//                                          k + 64, k the residual in units of 2^(e' - 14),
-//                                          e' the exponent of hi raised to at least -113)
+//                                          (bits(u) - bits(hi) + 2^15 + 2^8) >> 9, so that
+//                                          u ~ the float with bits bits(hi) + 2^9 (lo - 64))
 //   partial[chunk] = sum of u^2            for ||u||_F of the listing's G.norm()
 //   non-finite u                           counted into the workspace header, which then
 //                                          reports MUON_ERR_NONFINITE (values propagate)

@@ -8,8 +8,9 @@ in bfloat16 as the README's list of practices prescribes; the hi + lo carry of X
 library's reading of that practice):
 
   * u is fp32.  X is carried as hi = bf16(x) (round to nearest even) plus an 8-bit
-    fixed-point residual: with e' the exponent of hi raised to at least -113, the residual is
-    k = round-half-even((x - hi) 2^(14 - e')), and the carried value is hi + k 2^(e' - 14).
+    fixed-point residual on the fp32 bit patterns: with d = bits(x) - bits(hi), the residual
+    is k = floor((d + 2^8) / 2^9), and the carried value is the float with bits
+    bits(hi) + 2^9 k.
   * s = 1 / (||u||_F + eps) in fp32.
   * Gram:        A = bf16(fp32(hi hi^T) * fp32(s^2))   (s^2 in iteration 0 only)
   * polynomial:  B = bf16(fma(c, fp32(A A), fp32(b A)))
@@ -37,19 +38,18 @@ def f32(x):
     return np.asarray(x, np.float64).astype(np.float32).astype(np.float64)
 
 
-def _exponent_unit(hi):
-    """2^(e' - 14) for each bf16 value hi, e' its unbiased exponent raised to at least -113."""
-    E = (np.asarray(hi, np.float32).view(np.uint32) >> 23) & 0xFF
-    return np.ldexp(1.0, np.maximum(E.astype(np.int64), 14) - 127 - 14)
+def _bits(x):
+    return np.asarray(x, np.float32).view(np.int32).astype(np.int64)
 
 
 def carry(x):
-    """(hi, the carried value hi + lo) of the fp32 values x."""
+    """(hi, the carried value) of the fp32 values x: the residual kept as k = floor((d + 2^8)
+    / 2^9) on d = bits(x) - bits(hi), the carried value the float with bits bits(hi) + 2^9 k."""
     x = f32(x)
     hi = bf16(x)
-    unit = _exponent_unit(hi)
-    k = np.rint((x - hi) / unit)  # exact quotient; np.rint rounds half to even
-    return hi, hi + k * unit
+    k = np.floor_divide(_bits(x) - _bits(hi) + 256, 512)
+    carried = (_bits(hi) + 512 * k).astype(np.int32).view(np.float32).astype(np.float64)
+    return hi, carried
 
 
 def newton_schulz(G, coeffs, eps=1e-7):

@@ -26,22 +26,19 @@ def ws_matrix(ws_buf, offset, rows, cols, ld, dtype=torch.bfloat16):
     return raw.view(dtype).reshape(rows, ld)[:, :cols].float()
 
 
-def lo8_unit(hi):
-    """2^(e' - 14) per element for a bf16-valued tensor hi, with e' its exponent raised to at
-    least -113 (biased 14) -- the unit of the 8-bit lo part (include/muon_b200.h)."""
-    E = (hi.float().contiguous().view(torch.int32) >> 23) & 0xFF
-    # built from exponent bits: exactly 2^(e' - 14) (a pow() may be off in the last bit,
-    # which moves exact ties of the rounding)
-    return ((E.clamp(min=14) - 14) << 23).to(torch.int32).view(torch.float32).double().where(
-        E > 14, torch.full_like(E, 2.0 ** -127, dtype=torch.float64))
+def bits32(x):
+    """fp32 bit patterns of a float tensor, as int64 (signed, so differences are exact)."""
+    return x.float().contiguous().view(torch.int32).long()
 
 
 def ws_lo8(ws_buf, offset, rows, cols, ld_bytes, hi):
-    """The 8-bit lo part of X inside the workspace, as fp64 values (k * 2^(e' - 14)), and the
-    residual integers k (stored byte - 64)."""
+    """The 8-bit lo part of X inside the workspace (include/muon_b200.h): the stored bytes
+    minus 64, k, and the value hi + lo they encode, as fp64 -- the float whose bit pattern
+    is bits(hi) + 2^9 k."""
     raw = ws_buf[offset: offset + rows * ld_bytes].view(torch.uint8).reshape(rows, ld_bytes)[:, :cols]
-    k = raw.double() - 64.0
-    return k * lo8_unit(hi), k
+    k = raw.long() - 64
+    x = (bits32(hi) + k * 512).to(torch.int32).view(torch.float32).double()
+    return x - hi.double(), k
 
 
 def ws_scalar(ws_buf, offset):

@@ -8,7 +8,7 @@ at one kernel (elementwise, Gram, polynomial or apply) and one orientation.
 import numpy as np
 import pytest
 
-from tests.gpu_util import lo8_unit, require_gpu, rel_fro, to_np, torch, ws_lo8, ws_matrix, ws_scalar
+from tests.gpu_util import bits32, require_gpu, rel_fro, to_np, torch, ws_lo8, ws_matrix, ws_scalar
 
 pytestmark = pytest.mark.gpu
 
@@ -74,18 +74,19 @@ def test_one_iteration_stage_by_stage(shape):
     # elementwise: hi = bf16(G) and lo = the 8-bit residual, exactly as the format states
     Gd = G.double()
     assert torch.equal(hi, G.to(torch.bfloat16).float())
-    _, q = ws_lo8(ws.buf, view.x_lo_offset, rows, cols, view.x_lo_ld, hi)
-    unit = lo8_unit(hi)
-    q_ref = torch.round((Gd - hi.double()) / unit)  # round half to even; exact division by 2^k
+    lo_val, q = ws_lo8(ws.buf, view.x_lo_offset, rows, cols, view.x_lo_ld, hi)
+    d = bits32(G) - bits32(hi)  # |d| <= 2^15: rounding to bf16 rounds the bit pattern
+    assert d.abs().max().item() <= 2 ** 15
+    q_ref = torch.div(d + 256, 512, rounding_mode="floor")  # d rounded to a multiple of 2^9, halves up
     assert q_ref.abs().max().item() <= 64
     bad = q != q_ref
     if bad.any():
         i, j = [int(v) for v in bad.nonzero()[0]]
-        raise AssertionError(f"8-bit lo differs from round-half-even((x - hi) / 2^(e' - 14)) at {int(bad.sum())} "
-                             f"elements, first ({i}, {j}): got {float(q[i, j])} want {float(q_ref[i, j])}, "
-                             f"x {float(Gd[i, j])!r} hi {float(hi[i, j])!r} unit {float(unit[i, j])!r}")
-    # x = hi + k 2^(e' - 14) is within 2^(e - 15) <= 2^-15 |hi| of the fp32 input
-    assert ((hi.double() + q * unit) - Gd).abs().le(2 ** -15 * hi.double().abs() + 1e-38).all()
+        raise AssertionError(f"8-bit lo differs from (bits(x) - bits(hi) + 2^8) >> 9 at {int(bad.sum())} "
+                             f"elements, first ({i}, {j}): got {int(q[i, j])} want {int(q_ref[i, j])}, "
+                             f"x {float(Gd[i, j])!r} hi {float(hi[i, j])!r}")
+    # the float with bits bits(hi) + 2^9 k is within 2^8 fp32 ulps (2^-15 relative) of the input
+    assert ((hi.double() + lo_val) - Gd).abs().le(2 ** -15 * Gd.abs() + 1e-38).all()
     assert abs(nrm - Gd.norm().item()) <= 1e-6 * Gd.norm().item()
     assert abs(s - 1.0 / (Gd.norm().item() + 1e-7)) <= 1e-6 * s
 
