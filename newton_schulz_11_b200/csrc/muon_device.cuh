@@ -207,6 +207,16 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
+// The same without release semantics: orders nothing but the arrival itself.  For a signal
+// that only hands a tensor-memory accumulator back to the MMA issuer: the arriving threads
+// have completed their tensor-memory loads (tcgen05.wait::ld) and fenced them
+// (tcgen05.fence::before_thread_sync), and the waiter reads none of their ordinary memory
+// writes.  A release arrive would also wait for this thread's earlier global stores.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+
 // Pair TMA load: the box lands in this CTA's shared memory and its bytes complete
 // on the mbarrier at `bar_cluster` (the leader CTA's).  No multicast.
 __device__ __forceinline__ void tma_load_3d_pair(void* smem_dst, const CUtensorMap* map, uint32_t bar_cluster,

@@ -526,14 +526,15 @@ muon_status_t build_wave(const muon_matrix_t* mats, const WavePlan& w, uint8_t* 
   for (int cur = 0; cur < 2; ++cur) {
     GemmParams g = base;
     GemmParams a = base;
-    g.staged = kStreamed;
+    g.staged = kStreamed;  // (five 64-deep stages measured no faster than three 128-deep ones)
     a.staged = staged ? kStaged : kStreamed;
     for (int k = 0; k < nc; ++k) {
       const int ci = ord_sym[k];
       g.cls[k] = sym[ci];
       g.cls[k].ksize = static_cast<int32_t>(w.classes[ci].n);
       g.cls[k].a_mn = g.cls[k].b_mn = w.classes[ci].tall;
-      g.map_a[k] = g.map_b[k] = op_hi[ci][cur];
+      // 64-deep k-blocks of MN-major (tall) operands load 64 x 64 boxes
+      g.map_a[k] = g.map_b[k] = (g.staged == kStaged && w.classes[ci].tall) ? st_hi[ci][cur] : op_hi[ci][cur];
       g.map_out[k] = st_a[ci];
 
       const int cj = ord_app[k];

@@ -69,10 +69,19 @@ struct Lay {
   static constexpr bool kSym = MODE == kGram || MODE == kPoly;
   static constexpr bool SMALL = VAR == kStaged;
   static constexpr bool kLoader = SMALL && !kSym;  // staged applies: a warp stages the epilogue's inputs
+  // staged applies: 64-column quarters of the tile's old hi (16 KB) and lo (8 KB) in flight
+  // (four stages and four slots measured faster than five and two, or six and one)
+  static constexpr int kSlots = kLoader ? 4 : 0;
+  static constexpr int kSlotBytes = 3 * kBM * 64;  // 24 KB
   static constexpr int TM = 256;  // pair tile rows (128 per CTA)
   static constexpr int TN = 256;  // pair tile columns = UMMA N
   static constexpr int BK = VAR == kStreamed ? 128 : 64;
-  static constexpr int S = !SMALL ? 3 : (MODE == kGram ? 5 : (kSym ? 3 : 4));
+#ifndef MUON_POLY_OUTBUFS
+#define MUON_POLY_OUTBUFS 2
+#endif
+  // staged symmetric products: output staging buffers (32 KB each)
+  static constexpr int kOutBufs = MODE == kPoly ? MUON_POLY_OUTBUFS : 2;
+  static constexpr int S = !SMALL ? 3 : (MODE == kGram ? 5 : (kSym ? (kOutBufs == 1 ? 4 : 3) : 4));
   // epilogue warps (16 for the staged apply measured no faster than 8)
   static constexpr int NEPI = 8;
   static constexpr int kBox64 = 64 * 64 * 2;       // one 64 x 64 box: 8 KB
@@ -83,7 +92,8 @@ struct Lay {
   static constexpr int kRing = S * kStageBytes;
   // streamed: one 64-column quarter of this CTA's 128 x 256 tile at a time (symmetric
   // modes D_q and T_q, apply hi_q and lo_q); staged: see above
-  static constexpr int kEpi = !SMALL ? 2 * kHalf : (MODE == kGram ? 4 * kHalf : (kSym ? 8 * kHalf : 6 * kHalf));
+  static constexpr int kEpi = !SMALL ? 2 * kHalf
+                                     : (MODE == kGram ? 4 * kHalf : (kSym ? (4 + 2 * kOutBufs) * kHalf : kSlots * kSlotBytes));
   static constexpr int kBarOff = kRing + kEpi;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;
   static constexpr int kEpiThreads = 32 * NEPI;
@@ -91,6 +101,7 @@ struct Lay {
   static constexpr int kThreads = 64 + kEpiThreads + (kLoader ? 32 : 0);
   static constexpr int kTmemCols = 2 * TN;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(S <= 8, "barrier area");
 };
 
 template <int MODE>
@@ -206,15 +217,11 @@ __device__ __forceinline__ uint32_t region_chunk(int r, int c16) {
   return static_cast<uint32_t>((((r >> 6) * 4 + (c16 >> 3)) << 13) + rr * 128 + (((c16 & 7) ^ (rr & 7)) << 4));
 }
 
-// TMA transfers of the staged region's column boxes [cb0, cb0 + ncb) at rows row0..,
-// columns col0.. of matrix `mat`.  Parts outside the matrix are read as zero and not written.
-__device__ __forceinline__ void store_region(const CUtensorMap* map, const uint8_t* buf, int cb0, int ncb, int row0,
-                                             int col0, int mat) {
-#pragma unroll 1
-  for (int rb = 0; rb < 2; ++rb)
-#pragma unroll 1
-    for (int cb = cb0; cb < cb0 + ncb; ++cb)
-      tma_store_3d(map, buf + ((4 * rb + cb) << 13), col0 + 64 * cb, row0 + 64 * rb, mat);
+// A staged 128-row x 64-column bf16 quarter, two 64 x 64 boxes (rows 0-63, then 64-127) in the
+// same swizzle: row r's 16-byte chunk c (0..7).
+__device__ __forceinline__ uint32_t quarter_chunk(int r, int c16) {
+  const int rr = r & 63;
+  return static_cast<uint32_t>(((r >> 6) << 13) + rr * 128 + ((c16 ^ (rr & 7)) << 4));
 }
 
 // Loads column box cb (both row boxes) of the staged region.
@@ -323,7 +330,6 @@ __device__ __forceinline__ void store_lo32(uint8_t* row, int valid, bool v8, con
   }
 }
 
-constexpr int kLoBlock = kBM * 64;  // one quarter of 8-bit lo: 128 rows x 64 bytes
 
 // A staged 128-row x 64-byte block of the 8-bit lo buffer (one TMA box, 64-byte swizzle):
 // row r at r * 64 B, its 16-byte chunk c (0..3) at chunk c ^ ((r >> 1) & 3).
@@ -750,55 +756,60 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, VAR>::kThr
     }
   } else if (L::kLoader && warp == L::kLoaderWarp) {
     // ---------------------------------------------------------------- epilogue input loader (both CTAs)
-    // Quarter q of tile k's old hi and lo (this CTA's 128 rows x 64 columns) is loaded into
-    // its staging slot once every epilogue warp has read quarter q of tile k - 1.
+    // The quarters of this pair's tiles, in order (quarter g = 4 k + q of the k-th tile), go
+    // to slot g % kSlots: this CTA's 128 rows x 64 columns of the old hi and lo, loaded once
+    // every epilogue warp has read quarter g - kSlots from that slot.  (Prefetching the next
+    // tile's quarters into L2 at the start of each tile measured slower.)
     if (lane == 0) {
-      uint8_t* hib = epi;
-      uint8_t* lob = epi + 4 * L::kHalf;
+      constexpr int NS = L::kSlots > 0 ? L::kSlots : 1;  // (this branch runs in the staged applies only)
       int k = 0;
+      uint32_t g = 0;
       bool ok = true;
-      uint32_t issued = 0, last_par = 0;  // per quarter: a load issued; the parity of the last one
+      uint32_t issued = 0, last_par = 0;  // per slot: a load issued; the parity of the last one
       for (int t = pair; ok && t < p.total_tiles; t += npairs, ++k) {
         const Tile tl = decode_tile<MODE>(p, t);
         const int row0 = L::TM * tl.I + kBM * rank, col0 = L::TN * tl.J;
-        for (int q = 0; q < 4; ++q) {
-          if (k > 0 && !mbar_wait(&consumed[q], static_cast<uint32_t>(k - 1) & 1u, wd, kSiteProducerEpi)) {
+        for (int q = 0; q < 4; ++q, ++g) {
+          const int sl = static_cast<int>(g % NS);
+          if (g >= static_cast<uint32_t>(NS) &&
+              !mbar_wait(&consumed[sl], ((g / NS) - 1u) & 1u, wd, kSiteProducerEpi)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&efull[q], L::kHalf + kLoBlock);
-          load_region_quarter(hib, &p.map_in[tl.cls], &efull[q], q, row0, col0, tl.mat);
-          tma_load_3d(lob + q * kLoBlock, &p.map_out2[tl.cls], &efull[q], col0 + 64 * q, row0, tl.mat);
-          issued |= 1u << q;
-          last_par = (last_par & ~(1u << q)) | ((static_cast<uint32_t>(k) & 1u) << q);
+          uint8_t* slot = epi + sl * L::kSlotBytes;
+          mbar_arrive_expect_tx(&efull[sl], L::kSlotBytes);
+          tma_load_3d(slot, &p.map_in[tl.cls], &efull[sl], col0 + 64 * q, row0, tl.mat);
+          tma_load_3d(slot + L::kBox64, &p.map_in[tl.cls], &efull[sl], col0 + 64 * q, row0 + 64, tl.mat);
+          tma_load_3d(slot + 2 * L::kBox64, &p.map_out2[tl.cls], &efull[sl], col0 + 64 * q, row0, tl.mat);
+          issued |= 1u << sl;
+          last_par = (last_par & ~(1u << sl)) | (((g / NS) & 1u) << sl);
         }
       }
-      // Before the CTA leaves, every load issued has landed.  A quarter has at most one load
+      // Before the CTA leaves, every load issued has landed.  A slot has at most one load
       // outstanding: the one before it was waited for by every epilogue warp.
-      for (int q = 0; q < 4; ++q)
-        if (issued & (1u << q)) quiet_wait(&efull[q], (last_par >> q) & 1u, tb);
+      for (int sl = 0; sl < NS; ++sl)
+        if (issued & (1u << sl)) quiet_wait(&efull[sl], (last_par >> sl) & 1u, tb);
     }
   } else if constexpr (SMALL && !kSym) {
     // ---------------------------------------------------------------- staged apply epilogue (both CTAs)
-    // The tile's old hi and lo (128 x 256 each per CTA) arrive in shared memory as four
-    // 64-column quarters from the loader warp.  Each warp waits for the accumulator and each
-    // quarter itself, reads its part, tells the loader it is done with the quarter, and
-    // writes its results straight to global memory: the new pair (kApply) or W and/or O
-    // (kApplyLast).  The epilogue warps never wait for one another.
+    // The tile's old hi and lo (128 x 256 each per CTA) arrive in shared memory as 64-column
+    // quarters from the loader warp, quarter g of this pair's sequence in slot g % kSlots.
+    // Each warp waits for the accumulator and each quarter itself, reads its part, tells the
+    // loader it is done with the slot, and writes its results straight to global memory:
+    // the new pair (kApply) or W and/or O (kApplyLast).  The epilogue warps never wait for
+    // one another.
     const int ew = warp - 2;
     const int q4 = warp & 3;  // TMEM lanes 32 q4 .. 32 q4 + 31 belong to this warp
     const int h = ew >> 2;    // which 32 columns of each 64-column quarter
     const int r = q4 * 32 + lane;
     const uint32_t tempty0 = map_to_rank(smem_u32(tempty), 0);
-    uint8_t* hib = epi;
-    uint8_t* lob = epi + 4 * L::kHalf;
+    constexpr int NS = L::kSlots;
     int acc = 0;
     uint32_t aph = 0;
-    int k = 0;
-    for (int t = pair; t < p.total_tiles; t += npairs, ++k) {
+    uint32_t g = 0;  // quarters of this pair's tiles so far
+    for (int t = pair; t < p.total_tiles; t += npairs) {
       const Tile tl = decode_tile<MODE>(p, t);
       const ClassDesc& cd = p.cls[tl.cls];
-      const uint32_t kpar = static_cast<uint32_t>(k) & 1u;
       const int Rx = L::TM * tl.I + kBM * rank + r;
       const bool live = Rx < cd.rows;
       const bool hv8 = (cd.ldx & 15) == 0, lv8 = (cd.ldl & 31) == 0;  // 32-byte rows
@@ -827,9 +838,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, VAR>::kThr
       bool ok = warp_wait(&tfull[acc], aph, wd, kSiteEpilogueFull);
       if (ok) tc_fence_after();
 #pragma unroll 1
-      for (int q = 0; ok && q < 4; ++q) {
-        ok = warp_wait(&efull[q], kpar, wd, kSiteEpilogueIn);
+      for (int q = 0; ok && q < 4; ++q, ++g) {
+        const int sl = static_cast<int>(g % NS);
+        ok = warp_wait(&efull[sl], (g / NS) & 1u, wd, kSiteEpilogueIn);
         if (!ok) break;
+        const uint8_t* slot = epi + sl * L::kSlotBytes;
         const int c0 = 64 * q + 32 * h;
         uint4 wn[4];
         bool wn_ok = false;
@@ -838,8 +851,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, VAR>::kThr
         tmem_ld_32x32b_x32(tacc + c0, v);
         uint4 xh4[4], xl4[2];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) xh4[i] = *reinterpret_cast<const uint4*>(hib + region_chunk(r, (c0 >> 3) + i));
-        const uint8_t* lq = lob + (q << 13);
+        for (int i = 0; i < 4; ++i) xh4[i] = *reinterpret_cast<const uint4*>(slot + quarter_chunk(r, 4 * h + i));
+        const uint8_t* lq = slot + 2 * L::kBox64;
 #pragma unroll
         for (int i = 0; i < 2; ++i) xl4[i] = *reinterpret_cast<const uint4*>(lq + lo8_chunk(r, 2 * h + i));
         float x[32];
@@ -848,13 +861,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, VAR>::kThr
         // The slot may be refilled once every warp's reads of it have completed: the decode
         // above consumed the loaded values, and the proxy fence orders these generic-proxy
         // reads before the loader's TMA (async-proxy) write of the next tile's quarter.
+        // (Without the fence the loader's refill was measured to race these reads.)
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&consumed[q]);  // this warp is done with quarter q
+        if (lane == 0) mbar_arrive(&consumed[sl]);  // this warp is done with the slot
         if (q == 3) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * static_cast<uint32_t>(acc));
+          if (lane == 0) mbar_arrive_cluster_relaxed(tempty0 + 8u * static_cast<uint32_t>(acc));
         }
 #pragma unroll
         for (int j = 0; j < 32; ++j) x[j] = fmaf(p.a, x[j], __uint_as_float(v[j]));
@@ -895,7 +909,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, VAR>::kThr
     const int r = q4 * 32 + lane;
     const bool leader = threadIdx.x == 64;  // also the thread that waits on the barriers
     const uint32_t tempty0 = map_to_rank(smem_u32(tempty), 0);
-    uint8_t* Ain = epi + 4 * L::kHalf;
+    uint8_t* Ain = epi + 2 * L::kOutBufs * L::kHalf;
     int acc = 0;
     uint32_t aph = 0;
     uint32_t pending = 0, pend_par = 0;
@@ -906,7 +920,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, VAR>::kThr
       pending |= 1u << q;
       pend_par = (pend_par & ~(1u << q)) | (par << q);
     };
-    if (MODE == kPoly && leader && pair < p.total_tiles) {
+    constexpr bool kStageA = MODE == kPoly;
+    if (kStageA && leader && pair < p.total_tiles) {
       const Tile first = decode_tile<MODE>(p, pair);
       for (int q = 0; q < 4; ++q) load_quarter(first, q, 0u);
     }
@@ -932,11 +947,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, VAR>::kThr
         const bool skip = rb > cb;  // below the diagonal: stored by the block's mirror (uniform)
         if (ew == 0) {
           bool ok = q > 0 || warp_wait(&tfull[acc], aph, wd, kSiteEpilogueFull);
-          if (MODE == kPoly && ok) ok = warp_wait(&efull[q], kpar, wd, kSiteEpilogueIn);
+          if (kStageA && ok) ok = warp_wait(&efull[q], kpar, wd, kSiteEpilogueIn);
           if (lane == 0) {
             *epi_flag = ok ? 1 : 0;
             if (ok) pending &= ~(1u << q);
-            if (!skip) bulk_wait_read<1>();  // the stores that used this buffer last have read it
+            if (!skip) {  // the stores that used this buffer last have read it
+              if constexpr (L::kOutBufs == 1) bulk_wait_read<0>();
+              else bulk_wait_read<1>();
+            }
           }
         }
         named_barrier(1, NT);
@@ -946,7 +964,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, VAR>::kThr
         }
         if (q == 0) tc_fence_after();
         if (!skip) {
-          uint8_t* Q = epi + (used & 1u) * (2 * L::kHalf);
+          uint8_t* Q = epi + (L::kOutBufs == 1 ? 0u : (used & 1u)) * (2 * L::kHalf);
           uint8_t* Tst = Q + L::kHalf;
           uint4 ain[4];
 #pragma unroll
@@ -966,9 +984,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, VAR>::kThr
         if (q == 3) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * static_cast<uint32_t>(acc));
+          if (lane == 0) mbar_arrive_cluster_relaxed(tempty0 + 8u * static_cast<uint32_t>(acc));
         }
-        if (MODE == kPoly && leader && has_next) load_quarter(nx, q, kpar ^ 1u);
+        if (kStageA && leader && has_next) load_quarter(nx, q, kpar ^ 1u);
       }
       if (!live) break;
       if (++acc == 2) {
@@ -1063,7 +1081,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, VAR>::kThr
           if (q == 3) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * static_cast<uint32_t>(acc));
+            if (lane == 0) mbar_arrive_cluster_relaxed(tempty0 + 8u * static_cast<uint32_t>(acc));
           }
           fence_proxy_async_smem();
           named_barrier(1, NT);
@@ -1089,7 +1107,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, VAR>::kThr
           if (q == 3) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * static_cast<uint32_t>(acc));
+            if (lane == 0) mbar_arrive_cluster_relaxed(tempty0 + 8u * static_cast<uint32_t>(acc));
           }
           if constexpr (MODE == kApply) {
             if (leader) bulk_wait_read<0>();
