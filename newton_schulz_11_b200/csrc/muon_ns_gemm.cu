@@ -76,13 +76,13 @@ struct Lay {
   static constexpr int TM = 256;  // pair tile rows (128 per CTA)
   static constexpr int TN = 256;  // pair tile columns = UMMA N
   static constexpr int BK = VAR == kStreamed ? 128 : 64;
-#ifndef MUON_POLY_OUTBUFS
-#define MUON_POLY_OUTBUFS 2
-#endif
-  // staged symmetric products: output staging buffers (32 KB each)
-  static constexpr int kOutBufs = MODE == kPoly ? MUON_POLY_OUTBUFS : 2;
+  // staged symmetric products: output staging buffers (32 KB each).  The polynomial takes
+  // one, and a fourth operand stage with the space (measured faster than two and three).
+  static constexpr int kOutBufs = MODE == kPoly ? 1 : 2;
   static constexpr int S = !SMALL ? 3 : (MODE == kGram ? 5 : (kSym ? (kOutBufs == 1 ? 4 : 3) : 4));
-  // epilogue warps (16 for the staged apply measured no faster than 8)
+  // epilogue warps; in the staged applies each handles 256 / NEPI columns of every quarter
+  // (16 warps, or the new hi/lo written back into the slot and stored by TMA from the
+  // loader warp, measured slower there)
   static constexpr int NEPI = 8;
   static constexpr int kBox64 = 64 * 64 * 2;       // one 64 x 64 box: 8 KB
   static constexpr int kHalf = kBM * kBox * 2;      // one 64 x 128 box: 16 KB
@@ -295,41 +295,47 @@ __device__ __forceinline__ void load_row32_u8(const uint8_t* row, int valid, boo
   }
 }
 
-// 32 consecutive bf16 of one row (16 words, element 2i in the low half of word i) to `row`,
-// the first `valid` of them only; v8: the segment is 32-byte aligned.
-__device__ __forceinline__ void store_hi32(__nv_bfloat16* row, int valid, bool v8, const uint32_t (&w)[16]) {
-  if (valid >= 32) {
+// NC (16 or 32) consecutive bf16 of one row (NC / 2 words, element 2i in the low half of
+// word i) to `row`, the first `valid` of them only; v8: the segment is 32-byte aligned.
+template <int NC>
+__device__ __forceinline__ void store_hi_n(__nv_bfloat16* row, int valid, bool v8, const uint32_t (&w)[NC / 2]) {
+  if (valid >= NC) {
     if (v8) {
-      st_global_v8(row, make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]));
-      st_global_v8(row + 16, make_uint4(w[8], w[9], w[10], w[11]), make_uint4(w[12], w[13], w[14], w[15]));
+#pragma unroll
+      for (int q = 0; q < NC / 16; ++q)
+        st_global_v8(row + 16 * q, make_uint4(w[8 * q], w[8 * q + 1], w[8 * q + 2], w[8 * q + 3]),
+                     make_uint4(w[8 * q + 4], w[8 * q + 5], w[8 * q + 6], w[8 * q + 7]));
     } else {
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
+      for (int q = 0; q < NC / 8; ++q)
         reinterpret_cast<uint4*>(row)[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
     }
   } else {
 #pragma unroll
-    for (int j = 0; j < 32; ++j)
+    for (int j = 0; j < NC; ++j)
       if (j < valid) put_bf16(row + j, (j & 1) ? (w[j >> 1] >> 16) : (w[j >> 1] & 0xFFFFu));
   }
 }
 
-// 32 stored residual bytes (8 words, element j in byte j % 4 of word j / 4), the first `valid`.
-__device__ __forceinline__ void store_lo32(uint8_t* row, int valid, bool v8, const uint32_t (&w)[8]) {
-  if (valid >= 32) {
-    if (v8) {
-      st_global_v8(row, make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]));
+// NC (16 or 32) stored residual bytes (NC / 4 words, element j in byte j % 4 of word j / 4),
+// the first `valid`; v8 (NC = 32): the segment is 32-byte aligned, else 16-byte aligned.
+template <int NC>
+__device__ __forceinline__ void store_lo_n(uint8_t* row, int valid, bool v8, const uint32_t (&w)[NC / 4]) {
+  if (valid >= NC) {
+    if (NC == 32 && v8) {
+      st_global_v8(row, make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4 % (NC / 4)], w[5 % (NC / 4)],
+                                                                       w[6 % (NC / 4)], w[7 % (NC / 4)]));
     } else {
-      reinterpret_cast<uint4*>(row)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-      reinterpret_cast<uint4*>(row)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+#pragma unroll
+      for (int q = 0; q < NC / 16; ++q)
+        reinterpret_cast<uint4*>(row)[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
     }
   } else {
 #pragma unroll
-    for (int j = 0; j < 32; ++j)
+    for (int j = 0; j < NC; ++j)
       if (j < valid) row[j] = static_cast<uint8_t>(w[j >> 2] >> (8 * (j & 3)));
   }
 }
-
 
 // A staged 128-row x 64-byte block of the 8-bit lo buffer (one TMA box, 64-byte swizzle):
 // row r at r * 64 B, its 16-byte chunk c (0..3) at chunk c ^ ((r >> 1) & 3).
@@ -800,7 +806,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, VAR>::kThr
     // one another.
     const int ew = warp - 2;
     const int q4 = warp & 3;  // TMEM lanes 32 q4 .. 32 q4 + 31 belong to this warp
-    const int h = ew >> 2;    // which 32 columns of each 64-column quarter
+    constexpr int NC = 256 / L::NEPI;  // columns of each quarter per thread
+    const int h = ew >> 2;             // which NC columns of each 64-column quarter
     const int r = q4 * 32 + lane;
     const uint32_t tempty0 = map_to_rank(smem_u32(tempty), 0);
     constexpr int NS = L::kSlots;
@@ -817,10 +824,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, VAR>::kThr
       const int64_t loff = tl.mat * cd.lo_stride + static_cast<int64_t>(Rx) * cd.ldl;
       const float sc = p.first_iter ? p.scale[cd.mat_base + tl.mat] : 1.f;
       const uint32_t tacc = tmem_base + static_cast<uint32_t>(acc * L::TN) + (static_cast<uint32_t>(q4 * 32) << 16);
-      uint4 wq[4];
+      uint4 wq[NC / 8];
       bool wq_ok = false;
       if constexpr (MODE == kApplyLast) {
-        wq_ok = load_w_segment<MODE, 32>(p, cd, tl, rank, r, 32 * h, wq);
+        wq_ok = load_w_segment<MODE, NC>(p, cd, tl, rank, r, NC * h, wq);
         if (h == 0 && t + npairs < p.total_tiles) {  // warm L2 with this thread's row of W in the next tile
           const Tile nx = decode_tile<MODE>(p, t + npairs);
           const ClassDesc& nd = p.cls[nx.cls];
@@ -843,20 +850,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, VAR>::kThr
         ok = warp_wait(&efull[sl], (g / NS) & 1u, wd, kSiteEpilogueIn);
         if (!ok) break;
         const uint8_t* slot = epi + sl * L::kSlotBytes;
-        const int c0 = 64 * q + 32 * h;
-        uint4 wn[4];
+        const int c0 = 64 * q + NC * h;
+        uint4 wn[NC / 8];
         bool wn_ok = false;
-        if constexpr (MODE == kApplyLast) wn_ok = q < 3 && load_w_segment<MODE, 32>(p, cd, tl, rank, r, c0 + 64, wn);
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tacc + c0, v);
-        uint4 xh4[4], xl4[2];
+        if constexpr (MODE == kApplyLast) wn_ok = q < 3 && load_w_segment<MODE, NC>(p, cd, tl, rank, r, c0 + 64, wn);
+        uint32_t v[NC];
+        tmem_ld_row<NC>(tacc + c0, v);
+        uint4 xh4[NC / 8], xl4[NC / 16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) xh4[i] = *reinterpret_cast<const uint4*>(slot + quarter_chunk(r, 4 * h + i));
+        for (int i = 0; i < NC / 8; ++i)
+          xh4[i] = *reinterpret_cast<const uint4*>(slot + quarter_chunk(r, (NC / 8) * h + i));
         const uint8_t* lq = slot + 2 * L::kBox64;
 #pragma unroll
-        for (int i = 0; i < 2; ++i) xl4[i] = *reinterpret_cast<const uint4*>(lq + lo8_chunk(r, 2 * h + i));
-        float x[32];
-        decode_row<32>(reinterpret_cast<const uint32_t*>(xh4), reinterpret_cast<const uint32_t*>(xl4), x);
+        for (int i = 0; i < NC / 16; ++i) xl4[i] = *reinterpret_cast<const uint4*>(lq + lo8_chunk(r, (NC / 16) * h + i));
+        float x[NC];
+        decode_row<NC>(reinterpret_cast<const uint32_t*>(xh4), reinterpret_cast<const uint32_t*>(xl4), x);
         tmem_wait_ld();  // before any other asm: v is written asynchronously until here
         // The slot may be refilled once every warp's reads of it have completed: the decode
         // above consumed the loaded values, and the proxy fence orders these generic-proxy
@@ -871,23 +879,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, VAR>::kThr
           if (lane == 0) mbar_arrive_cluster_relaxed(tempty0 + 8u * static_cast<uint32_t>(acc));
         }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) x[j] = fmaf(p.a, x[j], __uint_as_float(v[j]));
+        for (int j = 0; j < NC; ++j) x[j] = fmaf(p.a, x[j], __uint_as_float(v[j]));
         if (sc != 1.f) {  // iteration 0 only (uniform)
 #pragma unroll
-          for (int j = 0; j < 32; ++j) x[j] *= sc;
+          for (int j = 0; j < NC; ++j) x[j] *= sc;
         }
         if constexpr (MODE == kApply) {
-          uint32_t hb[16], lb[8];
+          uint32_t hb[NC / 2], lb[NC / 4];
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
+          for (int i = 0; i < NC / 4; ++i)
             split_hi_lo8x4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3], hb[2 * i], hb[2 * i + 1], lb[i]);
           const int C = L::TN * tl.J + c0;
-          store_hi32(cd.x_hi_next + xoff + C, live ? cd.cols - C : 0, hv8, hb);
-          store_lo32(cd.x_lo + loff + C, live ? cd.cols - C : 0, lv8, lb);
+          store_hi_n<NC>(cd.x_hi_next + xoff + C, live ? cd.cols - C : 0, hv8, hb);
+          store_lo_n<NC>(cd.x_lo + loff + C, live ? cd.cols - C : 0, lv8, lb);
         } else {
-          write_update<MODE, 32>(p, cd, tl, rank, r, c0, x, wq_ok ? wq : nullptr);
+          write_update<MODE, NC>(p, cd, tl, rank, r, c0, x, wq_ok ? wq : nullptr);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) wq[i] = wn[i];
+          for (int i = 0; i < NC / 8; ++i) wq[i] = wn[i];
           wq_ok = wn_ok;
         }
       }
