@@ -53,3 +53,46 @@ def test_work_model_is_orientation_free():
     assert bench.matrix_work(768, 3072) == bench.matrix_work(3072, 768)
     mw = bench.matrix_work(256, 1024)
     assert mw["gram"] == 256 * 256 * 1024 and mw["poly"] == 256 ** 3 and mw["apply"] == 2 * 256 * 256 * 1024
+
+
+def test_roofline_takes_the_bound_with_the_longer_floor_and_fixed_denominators():
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0, "bf16_tflops_sustained": 1200.0}
+    # 0.75 TFLOP and 6 GB in 1 ms: 750 TF/s (0.5 of the tensor peak), 6000 GB/s (1.0 of HBM)
+    r = bench.roofline_of(0.75e12, 6e9, 1.0, peaks, "measured")
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["frac"] == pytest.approx(1.0) and r["frac_hbm"] == pytest.approx(1.0)
+    assert r["frac_tensor"] == pytest.approx(0.5)
+    assert r["frac_tensor_of_sustained"] == pytest.approx(0.625)
+    assert r["frac_nominal"]["tensor"] == pytest.approx(750 / bench.NOMINAL_PEAKS["bf16_tflops"], abs=1e-4)
+    # the same kernel with a tenth of the bytes is tensor-bound, against the burst peak whatever the clocks
+    r = bench.roofline_of(0.75e12, 0.6e9, 1.0, peaks, "measured")
+    assert r["bound"] == "tensor" and r["peak"] == 1500.0 and r["frac"] == pytest.approx(0.5)
+    # no flops: HBM
+    assert bench.roofline_of(0, 3e9, 1.0, peaks, "measured")["bound"] == "hbm"
+
+
+def test_both_arms_print_the_same_config():
+    w = inputs.WORKLOADS["gpt2-124m-72-matrices"]
+    import types
+
+    args = types.SimpleNamespace(steps=20, warmup=5, parallel="auto")
+    for world in (1, 2, 8):
+        mode = bench.parallel_mode(args, world)
+        assert mode == ("single" if world == 1 else "sharded")
+        line = bench.base_line(w, world, mode, 1.0, args)
+        assert line["config"] == bench.config_of(w, world, mode)
+        assert line["scaling"] == "strong"
+    args.parallel = "replicas"
+    assert bench.base_line(w, 4, bench.parallel_mode(args, 4), 1.0, args)["scaling"] == "weak"
+
+
+def test_oracle_plan_takes_full_steps_within_budget_and_windows_beyond(monkeypatch):
+    w = inputs.scaled_workload(inputs.WORKLOADS["gpt2-124m-72-matrices"], [(32, 32), (32, 64), (64, 32)] * 2)
+    ow = bench.OracleWorkload(w)
+    monkeypatch.setattr(ow, "run", lambda idx: 0.01 * len(idx))  # 10 ms per matrix, no oracle run
+    plans, total, sample = ow.plan(5, 10.0)
+    assert all(p == list(range(6)) for p in plans) and "full step" in sample
+    plans, total, sample = ow.plan(5, 0.1)  # 20 ms per run: windows of matrices, taken cyclically
+    assert all(1 <= len(p) < 6 for p in plans)
+    assert plans[1][0] == (plans[0][-1] + 1) % 6
+    assert total == sum(ow.work(i) for i in range(6))
