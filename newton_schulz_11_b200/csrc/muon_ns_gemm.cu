@@ -59,19 +59,21 @@ namespace muon {
 //   k-blocks in 32 KB stages, and the epilogue's inputs moved by TMA through shared
 //   memory -- there tiles are short, and the epilogue, not the main loop, sets the pace.
 //     Gram        five stages; two 32 KB output staging buffers (stores of one quarter
-//                 drain while the next is written)
-//     polynomial  three stages; two output buffers; the tile's A block (64 KB) staged
-//     apply       four stages; the tile's old hi (64 KB) and 8-bit lo (32 KB) staged by the
-//                 loader warp; the new hi and lo (or W and O) written with 32-byte global
-//                 stores, so no epilogue warp waits for a store or for another warp
+//                 drain while the next is written); not used (the Gram streams)
+//     polynomial  four stages; one output buffer; the tile's A block (64 KB) staged
+//     apply       five stages (the last apply four); the tile's old hi and 8-bit lo staged
+//                 by the loader warp in 24 KB quarter slots, two (four); the new hi and lo
+//                 (or W and O) written with 32-byte global stores, so no epilogue warp
+//                 waits for a store or for another warp
 template <int MODE, int VAR = kStreamed>
 struct Lay {
   static constexpr bool kSym = MODE == kGram || MODE == kPoly;
   static constexpr bool SMALL = VAR == kStaged;
   static constexpr bool kLoader = SMALL && !kSym;  // staged applies: a warp stages the epilogue's inputs
-  // staged applies: 64-column quarters of the tile's old hi (16 KB) and lo (8 KB) in flight
-  // (four stages and four slots measured faster than five and two, or six and one)
-  static constexpr int kSlots = kLoader ? 4 : 0;
+  // staged applies: 64-column quarters of the tile's old hi (16 KB) and lo (8 KB) in flight.
+  // The apply takes a fifth operand stage in place of two of the four slots (measured
+  // faster); the last apply, whose epilogue also reads and writes W, keeps four of each.
+  static constexpr int kSlots = !kLoader ? 0 : MODE == kApply ? 2 : 4;
   static constexpr int kSlotBytes = 3 * kBM * 64;  // 24 KB
   static constexpr int TM = 256;  // pair tile rows (128 per CTA)
   static constexpr int TN = 256;  // pair tile columns = UMMA N
@@ -79,7 +81,7 @@ struct Lay {
   // staged symmetric products: output staging buffers (32 KB each).  The polynomial takes
   // one, and a fourth operand stage with the space (measured faster than two and three).
   static constexpr int kOutBufs = MODE == kPoly ? 1 : 2;
-  static constexpr int S = !SMALL ? 3 : (MODE == kGram ? 5 : (kSym ? (kOutBufs == 1 ? 4 : 3) : 4));
+  static constexpr int S = !SMALL ? 3 : (MODE == kGram ? 5 : (kSym ? (kOutBufs == 1 ? 4 : 3) : (MODE == kApply ? 5 : 4)));
   // epilogue warps; in the staged applies each handles 256 / NEPI columns of every quarter
   // (16 warps, or the new hi/lo written back into the slot and stored by TMA from the
   // loader warp, measured slower there)

@@ -359,6 +359,26 @@ def test_wide_4096_shapes_at_full_size_in_one_grouped_call():
         assert err <= TOL_O, (w.shapes[i], err)
 
 
+def test_wide_4096_192_matrices_full_step_as_benchmarked():
+    """The 4096-wide set at full size in the launch configuration the bench times: all 192
+    matrices (5.9 B parameters, two waves) in one muon_step on device-drawn inputs.  Sampled
+    matrices from both waves, one of each shape, are checked against the fp64 oracle:
+    momentum, O and the bf16 update."""
+    require_gpu()
+    free, _ = torch.cuda.mem_get_info()
+    w = inputs.WORKLOADS["wide-4096-192-matrices"]
+    if free < 100e9:
+        pytest.skip(f"needs about 90 GB of device memory, {free / 1e9:.0f} GB free")
+    from newton_schulz_11_b200 import api
+
+    samples = [0, 190, 191]  # 4096^2 (first wave), 4096 x 14336 and 14336 x 4096 (second wave)
+    ws_bytes = api.workspace_size(w.shapes)  # what muon_step sizes its workspace to
+    waves = {api.scratch_view(w.shapes, i, ws_bytes).wave for i in samples}
+    _sampled_step_check(w, samples=samples, coeffs=QUINTIC5)
+    torch.cuda.empty_cache()
+    assert len(w.shapes) == 192 and waves == {0, 1}
+
+
 def test_bf16_update_on_ragged_views_keeps_the_neighbours():
     """The last apply updates bf16 W with 256-bit, 128-bit or element accesses, by the
     alignment of W's rows.  Ragged shapes as strided views inside larger sentinel-filled
