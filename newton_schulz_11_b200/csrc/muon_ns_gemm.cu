@@ -104,6 +104,7 @@ struct Lay {
   static constexpr int kTmemCols = 2 * TN;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(S <= 8, "barrier area");
+  static_assert(TM == TN && kABytes == kBBytes, "diagonal tiles read one operand tile as both");
 };
 
 template <int MODE>
@@ -168,6 +169,27 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t) {
     r.I = q / cd.nb;
   }
   return r;
+}
+
+// A diagonal pair tile (I == J) of a symmetric product: each CTA's A rows are its B rows
+// (both operands are the same matrix through the same tensor map, and TM == TN), so the
+// stage holds one operand tile and the MMA reads it as both.
+template <int MODE>
+__device__ __forceinline__ bool is_diag_tile(const Tile& tl) {
+  return (MODE == kGram || MODE == kPoly) && tl.I == tl.J;
+}
+
+// This CTA's bytes in stage-load i (issue order) of pair `pair`; used only to settle the
+// loads left open after a timeout.
+template <int MODE, class L>
+__device__ uint32_t load_share_bytes(const GemmParams& p, int pair, int npairs, uint32_t i) {
+  for (int t = pair; t < p.total_tiles; t += npairs) {
+    const Tile tl = decode_tile<MODE>(p, t);
+    const uint32_t nk = static_cast<uint32_t>((p.cls[tl.cls].ksize + L::BK - 1) / L::BK);
+    if (i < nk) return is_diag_tile<MODE>(tl) ? L::kABytes : L::kStageBytes;
+    i -= nk;
+  }
+  return L::kStageBytes;
 }
 
 // One operand tile (128 MN x BK) into `dst`, completing on the leader CTA's mbarrier.
@@ -662,6 +684,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, VAR>::kThr
         const int nk = (cd.ksize + L::BK - 1) / L::BK;
         const int a0 = L::TM * tl.I + kBM * rank;
         const int b0 = L::TN * tl.J + kBM * rank;
+        const bool diag = is_diag_tile<MODE>(tl);
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1u, wd, kSiteProducerEmpty)) {
             ok = false;
@@ -669,11 +692,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, VAR>::kThr
           }
           uint8_t* sa = smem + s * L::kStageBytes;
           uint8_t* sb = sa + L::kABytes;
-          if (leader_cta) mbar_arrive_expect_tx(&full[s], 2 * L::kStageBytes);
+          if (leader_cta) mbar_arrive_expect_tx(&full[s], 2 * (diag ? L::kABytes : L::kStageBytes));
           const uint32_t fb = full0 + 8u * static_cast<uint32_t>(s);
           const int k0 = kb * L::BK;
           load_operand_pair<L::BK>(sa, ma, cd.a_mn, a0, k0, tl.mat, fb);
-          load_operand_pair<L::BK>(sb, mb, cd.b_mn, b0, k0, tl.mat, fb);
+          if (!diag) load_operand_pair<L::BK>(sb, mb, cd.b_mn, b0, k0, tl.mat, fb);
           ++issued;
           if (++s == S) {
             s = 0;
@@ -709,9 +732,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, VAR>::kThr
           const int st = static_cast<int>(i % S);
           const uint32_t par = (i / S) & 1u;
           if (i >= nl)
-            mbar_arrive_expect_tx(&full[st], L::kStageBytes);
+            mbar_arrive_expect_tx(&full[st], load_share_bytes<MODE, L>(p, pair, npairs, i));
           else if (i >= np)
-            mbar_complete_tx(&full[st], L::kStageBytes);
+            mbar_complete_tx(&full[st], load_share_bytes<MODE, L>(p, pair, npairs, i));
           quiet_wait(&full[st], par, tb);
         }
       }
@@ -728,6 +751,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, VAR>::kThr
           const ClassDesc& cd = p.cls[tl.cls];
           const int nk = (cd.ksize + L::BK - 1) / L::BK;
           const uint32_t idesc = idesc_bf16_f32(L::TM, L::TN, cd.a_mn, cd.b_mn);
+          const bool diag = is_diag_tile<MODE>(tl);
           if (!mbar_wait(&tempty[acc], aph ^ 1u, wd, kSiteMmaTmemEmpty)) break;
           tc_fence_after();
           const uint32_t dtm = tmem_base + static_cast<uint32_t>(acc * L::TN);
@@ -738,7 +762,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<MODE, VAR>::kThr
             }
             tc_fence_after();
             const uint32_t sa = smem_u32(smem + s * L::kStageBytes);
-            const uint32_t sb = sa + L::kABytes;
+            const uint32_t sb = diag ? sa : sa + L::kABytes;
 #pragma unroll
             for (int kk = 0; kk < L::BK / 16; ++kk)
               umma_bf16_pair(dtm, operand_desc<L::BK>(sa, cd.a_mn, kk), operand_desc<L::BK>(sb, cd.b_mn, kk), idesc,
