@@ -649,6 +649,66 @@ def measure_wide(local, peaks, peak_src, steps=5, warmup=3):
     return out
 
 
+def torch_comparator_step(w, grads, moms, params, coeffs):
+    """The same step in plain PyTorch, the way the pages' listing runs it: for each shape
+    class, the matrices stacked and every Newton-Schulz product a batched bf16 matmul
+    (torch.bmm, cuBLAS), with X kept in bf16 between iterations; momentum, Nesterov input
+    and update as torch elementwise ops.  A library comparator for timing on the same GPU:
+    it is neither the product path nor the parity reference (the oracle is).  Returns
+    step() and the stacked (g, m, W) per class (W updated in place)."""
+    import torch
+
+    groups = {}
+    for i, shp in enumerate(w.shapes):
+        groups.setdefault(tuple(shp), []).append(i)
+    cls = []
+    for (r, c), idx in groups.items():
+        cls.append((torch.stack([grads[i] for i in idx]), torch.stack([moms[i] for i in idx]),
+                    torch.stack([params[i] for i in idx]), r > c, math.sqrt(max(1.0, r / c))))
+
+    def step():
+        for g, m, p, tall, scale in cls:
+            m.mul_(w.beta).add_(g)
+            u = g.add(m, alpha=w.beta) if w.nesterov else m
+            X = u.bfloat16()
+            X = X / (torch.linalg.vector_norm(X, dim=(1, 2), keepdim=True) + 1e-7)
+            if tall:
+                X = X.mT
+            for a, b, c in coeffs:
+                A = X @ X.mT
+                B = b * A + c * (A @ A)
+                X = a * X + B @ X
+            if tall:
+                X = X.mT
+            p.mul_(1.0 - w.lr * w.weight_decay).add_(X.to(p.dtype), alpha=-w.lr * scale)
+
+    return step, cls
+
+
+def measure_torch_comparator(w, local, ms_ours, steps=20, warmup=5):
+    """Times torch_comparator_step on this GPU on the workload's own inputs."""
+    import torch
+
+    dev = torch.device("cuda", local)
+    step0 = inputs.first_step_index(w)
+    n = len(w.shapes)
+    step, _ = torch_comparator_step(w, [inputs.grad_torch(w, step0, i, dev) for i in range(n)],
+                                    [inputs.momentum_torch(w, i, dev) for i in range(n)],
+                                    [inputs.weight_torch(w, i, dev) for i in range(n)], load_coeffs(w))
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    ms_t = time_steps(step, steps, 1, dev)
+    alg, _ = step_flops(w)
+    del step
+    torch.cuda.empty_cache()
+    return {"impl": "plain PyTorch: bf16 torch.bmm per shape class (cuBLAS), X kept in bf16",
+            "ms_per_step": round(ms_t, 4), "steps": steps, "warmup": warmup,
+            "ns_tflops": round(alg / (ms_t * 1e-3) / 1e12, 1), "time_ratio_to_ours": round(ms_t / ms_ours, 2),
+            "note": "a library comparator on the same GPU and inputs; lower precision than this "
+                    "library's path (X rounded to bf16 every iteration) and not parity-checked"}
+
+
 def run_ours(args, world, rank, local):
     import ctypes
 
@@ -782,6 +842,8 @@ def run_ours(args, world, rank, local):
         cms, sample = oracle_baseline_ms(w)
         line["cpu_baseline"] = {"value": round(cms, 1), "unit": "ms", "cores": blas_threads(), "kind": "oracle",
                                 "sample": sample}
+    if world == 1 and mode == "single" and not args.no_torch:
+        line["torch_comparator"] = measure_torch_comparator(w, local, ms_step)
     if world == 1 and w.name == DEFAULT_WORKLOAD and not args.no_wide:
         del G, M, P, gs, ms, ps, step, ws
         torch.cuda.empty_cache()
@@ -1044,6 +1106,8 @@ def main():
                     help="sharded: waves of owned matrices (a wave's broadcasts overlap the next wave's step)")
     ap.add_argument("--no-wide", action="store_true",
                     help="skip the 4096-wide measurement added to the default workload's line")
+    ap.add_argument("--no-torch", action="store_true",
+                    help="skip the plain-PyTorch (cuBLAS bf16 bmm) comparator timed beside the step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

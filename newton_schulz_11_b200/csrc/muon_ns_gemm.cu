@@ -23,7 +23,8 @@
 // the diagonal is stored twice by TMA, as itself at (i, j) and transposed at (j, i);
 // a diagonal block keeps its upper triangle and mirrors it into the lower one; a
 // block below the diagonal is dropped.  Every element has one writer, and the stored
-// matrices are exactly symmetric.
+// matrices are exactly symmetric.  On a diagonal pair tile each CTA's A rows are its B
+// rows, so its stages hold one operand tile and the MMAs read it as both.
 //
 // A tall matrix (rows > cols) is never transposed in memory.  With Y the stored
 // matrix (X = Y^T) the same iteration reads  A = Y^T Y  (both operands MN-major)
