@@ -91,6 +91,27 @@ def test_newton_schulz_matches_oracle(shape):
     assert err <= TOL_O, f"{shape}: rel err {err:.3e}"
 
 
+# A short side of a few dozen against a long side of about a million, both odd-sized so
+# that tile rows, tile columns and the last k-block are all ragged: the wide one is a
+# single pair tile whose Gram reduction runs 15,625 64-deep k-blocks; each apply spreads
+# 3,907 column tiles over the SMs.  The tall one runs the mirrored recurrence the same way.
+EXTREME = [(40, 1_000_001), (999_999, 24)]
+
+
+@pytest.mark.parametrize("shape", EXTREME, ids=[f"{r}x{c}" for r, c in EXTREME])
+def test_newton_schulz_extreme_aspect_ratio(shape):
+    require_gpu()
+    from newton_schulz_11_b200 import api
+
+    w = inputs.scaled_workload(inputs.WORKLOADS["single-256x128-f32"], [shape])
+    G = inputs.grad_np(w, 0, 0)
+    O = api.newton_schulz([torch.from_numpy(G).cuda()], coeffs=QUINTIC5)[0]
+    ref = oracle.newton_schulz(G.astype(np.float64), QUINTIC5)
+    err = rel_fro(to_np(O), ref)
+    print(f"NS {shape}: rel err {err:.3e}")
+    assert err <= TOL_O, f"{shape}: rel err {err:.3e}"
+
+
 @pytest.mark.parametrize("shape", DEGENERATE, ids=[f"{r}x{c}" for r, c in DEGENERATE])
 def test_newton_schulz_single_singular_value(shape):
     require_gpu()
