@@ -73,7 +73,8 @@ struct Lay {
   static constexpr bool kLoader = SMALL && !kSym;  // staged applies: a warp stages the epilogue's inputs
   // staged applies: 64-column quarters of the tile's old hi (16 KB) and lo (8 KB) in flight.
   // The apply takes a fifth operand stage in place of two of the four slots (measured
-  // faster); the last apply, whose epilogue also reads and writes W, keeps four of each.
+  // faster); the last apply, whose epilogue also reads and writes W, keeps four of each
+  // (five and two measured 2.5% slower there).
   static constexpr int kSlots = !kLoader ? 0 : MODE == kApply ? 2 : 4;
   static constexpr int kSlotBytes = 3 * kBM * 64;  // 24 KB
   static constexpr int TM = 256;  // pair tile rows (128 per CTA)
