@@ -211,6 +211,58 @@ def test_single_256x128_f32_step():
     assert rel_fro(dW_gpu, W_ref - W) <= TOL_O
 
 
+# The step's other options against the oracle: Nesterov off, beta 0, one, two and sixteen
+# iterations (the table's maximum; the classical cubic, which converges, since sixteen
+# quintic steps amplify bf16 rounding to about 3.5e-2 in the rounding model), an eps that
+# matters, an explicit shape scale, fp32 and bf16 W, wide, tall and square-ish shapes.
+CUBIC = (1.5, -0.5, 0.0)
+OPTION_CASES = [
+    # id, shape, W dtype, options
+    ("plain-momentum", (200, 136), "f32", dict(nesterov=False, beta=0.9, weight_decay=0.05, coeffs=[oracle.QUINTIC] * 5)),
+    ("beta0", (136, 200), "bf16", dict(nesterov=True, beta=0.0, weight_decay=0.0, coeffs=[oracle.QUINTIC] * 5)),
+    ("one-step", (300, 128), "f32", dict(nesterov=True, beta=0.95, weight_decay=0.1, coeffs=[oracle.QUINTIC])),
+    ("two-steps", (136, 200), "bf16", dict(nesterov=True, beta=0.95, weight_decay=0.0, coeffs=[oracle.QUINTIC] * 2)),
+    ("sixteen-steps", (200, 136), "f32", dict(nesterov=True, beta=0.95, weight_decay=0.0, coeffs=[CUBIC] * 16)),
+    ("eps-1e-3", (136, 200), "f32", dict(nesterov=True, beta=0.95, weight_decay=0.0, coeffs=[oracle.QUINTIC] * 5,
+                                         eps=1e-3, grad_scale=1e-6)),  # eps moves O by 5.9%
+    ("shape-scale", (300, 128), "bf16", dict(nesterov=True, beta=0.95, weight_decay=0.02, coeffs=[oracle.QUINTIC] * 5,
+                                              shape_scale=0.5)),
+]
+
+
+@pytest.mark.parametrize("case", OPTION_CASES, ids=[c[0] for c in OPTION_CASES])
+def test_step_options_match_the_oracle(case):
+    require_gpu()
+    from newton_schulz_11_b200 import api
+
+    _, shape, dtype, opt = case
+    opt = dict(opt)
+    eps = opt.pop("eps", oracle.NS_EPS)
+    gs_scale = opt.pop("grad_scale", 1.0)
+    scale = opt.pop("shape_scale", None)
+    w = inputs.scaled_workload(inputs.WORKLOADS["single-256x128-f32"], [shape])
+    g = (inputs.grad_np(w, 0, 0) * np.float32(gs_scale)).astype(np.float32)
+    m = (inputs.momentum_np(w, 0) * np.float32(gs_scale)).astype(np.float32)
+    W = inputs.weight_np(w, 0)
+    if dtype == "bf16":
+        W = inputs.bf16_round_np(W)
+    Wt, gt, mt = gpu_tensors(W, g, m, dtype)
+    O = torch.empty_like(gt)
+    lr = 0.02
+    api.muon_step([Wt], [gt], [mt], lr=lr, eps=eps, outs=[O], shape_scales=None if scale is None else [scale], **opt)
+    W_ref, m_ref, O_ref = oracle.muon_step(W.astype(np.float64), g, m, lr=lr, shape_scale=scale, eps=eps, **opt)
+    check_momentum(to_np(mt), m_ref, "momentum")
+    err = rel_fro(to_np(O), O_ref)
+    print(f"{case[0]} {shape}: O rel err {err:.3e}")
+    assert err <= TOL_O
+    s = oracle.default_shape_scale(*shape) if scale is None else scale
+    if dtype == "bf16":
+        check_bf16_update(to_np(Wt), W, to_np(O), lr, opt["weight_decay"], s, "W")
+    else:
+        W_from_O = oracle.parameter_update(W, to_np(O), lr, opt["weight_decay"], s)
+        assert rel_fro(to_np(Wt), W_from_O) <= TOL_F32
+
+
 def test_mlp_768x3072_bf16_three_steps():
     """768x3072 bf16 weight, momentum from zero, three steps on fresh grads, lr 0.05, wd 0.01."""
     require_gpu()
