@@ -8,7 +8,8 @@ device array inside the library (MUON_STATIC_SCRATCH_BYTES, held by every GPU th
 loads the library until exit).
 
 The GPU test calls the entry point through the C ABI twice in a row, on different
-inputs, and checks each result against the workspace entry point (muon_newton_schulz).
+inputs, and checks each result against the workspace entry point (muon_newton_schulz);
+each call is repeated through the Python binding, which must give the same bits.
 Both run the same kernels with the same per-matrix arithmetic in the same order, and
 the library's results do not depend on how matrices are grouped into waves, so the two
 must agree bit for bit (the workspace entry point is itself checked against the fp64
@@ -76,3 +77,11 @@ def test_static_scratch_matches_workspace_entry_point_on_two_calls():
             assert np.isfinite(o_np).all(), (r, c)
             assert torch.equal(o, o_ref), ((r, c), rel_fro(o_np, ref_np))
             assert rel_fro(o_np, ref_np) <= TOL_NS
+        # the Python binding of the same entry point: the same bits
+        outs2 = [torch.full_like(g, float("nan")) for g in Gs]
+        status.fill_(-1)
+        api.newton_schulz_static(Gs, outs=outs2, device_status=status)
+        torch.cuda.synchronize()
+        assert status.tolist() == [0, 0]
+        for o, o2 in zip(outs, outs2):
+            assert torch.equal(o, o2)
