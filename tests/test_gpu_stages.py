@@ -18,6 +18,7 @@ SHAPES = [
     (200, 136), (136, 200),                  # ragged tails (multiples of 8)
     (40, 72), (72, 40),                      # single partial tile
     (100, 37), (37, 100),                    # sides that are not multiples of 8
+    (600, 704), (704, 600),                  # three diagonal pair tiles, the last ragged (staged)
     (1048, 1152), (1152, 1048),              # Gram side above 1024: the streamed variant
 ]
 
