@@ -25,7 +25,9 @@
  *
  * Ownership: the caller allocates and owns every buffer, including the workspace,
  * and keeps them alive until the work queued on `stream` has finished.  The library
- * allocates no device memory.  `param` and `momentum` are updated in place; `grad`
+ * allocates no device memory; the one exception is the fixed static array that
+ * muon_newton_schulz_static works in, which the module holds on every GPU that loads
+ * it (MUON_STATIC_SCRATCH_BYTES).  `param` and `momentum` are updated in place; `grad`
  * is only read.  Buffers of different roles (and of different matrices) must not
  * overlap.  All device pointers must belong to the current CUDA device.
  *
