@@ -273,8 +273,9 @@ muon_status_t muon_adamw_step(const muon_adamw_tensor_t* tensors, int n, float l
  *     overlap on the GPU (other streams, other host threads) race on the array and
  *     give wrong results: keep them ordered, e.g. on one stream.
  *   - device_status (may be NULL): 2 int32 in device or pinned host memory; after the
- *     call's kernels, in stream order, it receives the status word (MUON_OK or
- *     MUON_ERR_TIMEOUT) and the wait that gave up, as muon_device_status reports them.
+ *     call's kernels, in stream order, it receives the status word (MUON_OK,
+ *     MUON_ERR_TIMEOUT or MUON_ERR_NONFINITE) and its `where`, as muon_device_status
+ *     reports them.
  */
 #define MUON_STATIC_SCRATCH_BYTES (64u << 20)
 
