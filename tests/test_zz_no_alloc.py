@@ -85,3 +85,22 @@ def test_static_scratch_matches_workspace_entry_point_on_two_calls():
         assert status.tolist() == [0, 0]
         for o, o2 in zip(outs, outs2):
             assert torch.equal(o, o2)
+
+
+@pytest.mark.gpu
+def test_static_scratch_reports_a_nonfinite_input():
+    """A NaN in one matrix's G: the status output reads MUON_ERR_NONFINITE with that
+    matrix's index, and the other matrix's O is still the workspace entry point's."""
+    from tests.gpu_util import require_gpu, torch
+
+    require_gpu()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    gen = torch.Generator(device=dev).manual_seed(13)
+    Gs = [torch.randn(256, 384, device=dev, generator=gen), torch.randn(192, 128, device=dev, generator=gen)]
+    Gs[1][5, 7] = float("nan")
+    status = torch.full((2,), -1, dtype=torch.int32, device=dev)
+    outs = api.newton_schulz_static(Gs, device_status=status)
+    ref = api.newton_schulz(Gs[:1], workspace=api.Workspace(dev))
+    torch.cuda.synchronize()
+    assert status.tolist() == [_lib.MUON_ERR_NONFINITE, 1]
+    assert torch.equal(outs[0], ref[0])
