@@ -187,6 +187,37 @@ def test_newton_schulz_grouped_mixed_shapes_and_schedule():
         assert err <= TOL_O, f"matrix {i} {shapes[i]}: {err:.3e}"
 
 
+def test_more_shape_classes_than_one_wave_holds():
+    """Twelve distinct shapes in one call: a wave holds at most eight shape classes, so the
+    call runs in two waves.  Every matrix matches the oracle, and equals the same matrix
+    stepped alone, bit for bit."""
+    require_gpu()
+    from newton_schulz_11_b200 import api
+
+    shapes = [(64, 64), (72, 40), (40, 72), (128, 96), (96, 128), (200, 136), (136, 200), (256, 64),
+              (64, 256), (100, 37), (37, 100), (160, 160)]
+    assert api.scratch_view(shapes, len(shapes) - 1, api.workspace_size(shapes)).wave == 1
+    w = inputs.scaled_workload(inputs.WORKLOADS["gpt2-124m-72-matrices"], shapes)
+    gs = [inputs.grad_np(w, 1, i) for i in range(len(shapes))]
+    ms = [inputs.grad_np(w, 0, i) for i in range(len(shapes))]
+    Ws = [inputs.bf16_round_np(inputs.weight_np(w, i)) for i in range(len(shapes))]
+    grouped = [gpu_tensors(W, g, m, "bf16") for W, g, m in zip(Ws, gs, ms)]
+    outs = [torch.empty_like(t[1]) for t in grouped]
+    api.muon_step([t[0] for t in grouped], [t[1] for t in grouped], [t[2] for t in grouped], lr=w.lr,
+                  beta=w.beta, weight_decay=0.01, coeffs=QUINTIC5, outs=outs)
+    for i, (W, g, m) in enumerate(zip(Ws, gs, ms)):
+        Wt, gt, mt = gpu_tensors(W, g, m, "bf16")
+        O = torch.empty_like(gt)
+        api.muon_step([Wt], [gt], [mt], lr=w.lr, beta=w.beta, weight_decay=0.01, coeffs=QUINTIC5, outs=[O])
+        for a, b in zip((Wt, mt, O), (grouped[i][0], grouped[i][2], outs[i])):
+            assert torch.equal(a, b), shapes[i]
+        _, m_ref, O_ref = oracle.muon_step(W.astype(np.float64), g, m, lr=w.lr, beta=w.beta, weight_decay=0.01,
+                                           nesterov=True, coeffs=QUINTIC5)
+        check_momentum(to_np(mt), m_ref, f"momentum {shapes[i]}")
+        err = rel_fro(to_np(O), O_ref)
+        assert err <= TOL_O, (shapes[i], err)
+
+
 # ----------------------------------------------------------------------- full steps
 
 def test_single_256x128_f32_step():
